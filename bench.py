@@ -1,0 +1,407 @@
+"""Benchmark of the mixed-precision routed-expert layer on B200.
+
+Headline workload: one Qwen3-30B-A3B-shaped MoE layer at decode batch 32
+(H=2048, I=768, E=128, top-8, Zipf(1.1) routing skew, the 32 hottest experts
+BF16 and the other 96 INT4 group-128).  A step is one whole layer forward
+(route -> permute -> grouped FFN -> combine) on one batch of 32 tokens; the
+same layer at prefill 4096 tokens (24 BF16 / 40 INT8 / 64 INT4 experts) is
+reported in the "prefill" object.  Inputs are seeded synthetic data with the
+shapes and value distributions of those workloads.
+
+Timing: each step is a CUDA-graph replay timed by CUDA events on the launching
+stream, with a 256 MiB write between steps to flush the 126 MB L2.  Multi-GPU
+runs are independent replicas (the layer does not shard): every rank runs the
+same workload and value = all ranks' tokens / the slowest rank's time.
+
+`--impl reference` times the CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixed_precision_moe_b200 import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at decode B=32 and prefill 4096; % HBM / BF16-tensor roofline"
+FLUSH_BYTES = 256 << 20
+
+
+def expert_bytes(prec, H, I):
+    """Stored bytes of one expert (weights + fp16 group-128 scales)."""
+    P = 3 * H * I
+    return {synth.BF16: 2 * P, synth.INT8: P + P // 64, synth.INT4: P // 2 + P // 64}[int(prec)]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def workload_name(cfg):
+    tiers = " + ".join(f"{n} {synth.PREC_NAMES[p].upper()}" for n, p in cfg.tiers)
+    return (f"{cfg.name}: H={cfg.H} I={cfg.I} E={cfg.E} top-{cfg.k} T={cfg.T}, "
+            f"Zipf({cfg.zipf_s}) routing, experts {tiers}")
+
+
+# --------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 6]
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[3:7]) if v.strip() == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------- our arm (GPU) --
+
+def build_layer(cfg, device):
+    """Experts from seeded bf16 masters; INT8/INT4 ones quantised on the GPU."""
+    from mixed_precision_moe_b200 import binding as B
+    ranks = synth.zipf_ranks(cfg.E, cfg.seed)
+    precs = synth.precision_map(ranks, cfg.tiers)
+    layer = B.MoELayer(cfg.H, cfg.I, cfg.E, cfg.k)
+    for e in range(cfg.E):
+        w13, w2 = synth.gen_expert_master(cfg.H, cfg.I, cfg.seed, e)
+        m13 = torch.from_numpy(w13.view(np.int16)).view(torch.bfloat16).to(device)
+        m2 = torch.from_numpy(w2.view(np.int16)).view(torch.bfloat16).to(device)
+        p = int(precs[e])
+        if p == synth.BF16:
+            layer.set_expert(e, p, m13, None, m2, None)
+        else:
+            q13, s13 = B.moe_quantize_weights(m13, p)
+            q2, s2 = B.moe_quantize_weights(m2, p)
+            layer.set_expert(e, p, q13, s13, q2, s2)
+    torch.cuda.synchronize()
+    return layer, ranks, precs
+
+
+def make_inputs(cfg, ranks, n_batches, device):
+    batches = []
+    for b in range(n_batches):
+        x = synth.gen_x(cfg.T, cfg.H, cfg.seed * 1000 + b)
+        lg = synth.gen_logits(cfg.T, cfg.E, cfg.seed * 1000 + b, cfg.zipf_s, ranks)
+        batches.append((torch.from_numpy(lg), torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)))
+    dev = [(lg.to(device), x.to(device)) for lg, x in batches]
+    return batches, dev
+
+
+def time_graphs(graphs, steps, warmup, flush, stream):
+    """Replay graphs[i % len] `steps` times after `warmup`; per-step event times (ms).
+    The flush, the replays and the events all go to `stream`."""
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            flush.zero_()
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            graphs[i % len(graphs)].replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def run_workload(cfg, steps, warmup, device, with_e2e, dist_barrier):
+    """Returns a dict of timings and accounting for one layer config."""
+    from mixed_precision_moe_b200 import binding as B
+    layer, ranks, precs = build_layer(cfg, device)
+    n_batches = 4
+    host_batches, dev_batches = make_inputs(cfg, ranks, n_batches, device)
+    stream = torch.cuda.Stream(device)
+    bufs = [layer.alloc_buffers(cfg.T, device) for _ in range(n_batches)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    # warm the library (attributes, tensor-map encoder) before capture
+    with torch.cuda.stream(stream):
+        for b in range(n_batches):
+            layer.forward(*dev_batches[b], bufs=bufs[b])
+    torch.cuda.synchronize()
+
+    step_graphs, ffn_graphs = [], []
+    for b in range(n_batches):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            layer.forward(*dev_batches[b], bufs=bufs[b], stream=stream)
+        step_graphs.append(g)
+        off, perm, dest, xp = bufs[b]["permute"]
+        y, ws = bufs[b]["ffn"]
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            B.moe_grouped_ffn_mixed(layer, xp, off, y, ws, stream=stream)
+        ffn_graphs.append(g2)
+    torch.cuda.synchronize()
+
+    # algorithmic accounting from this run's routing (read back after the fact)
+    touched_bytes, pairs, n_touched = [], [], []
+    for b in range(n_batches):
+        idx = bufs[b]["route"][0].cpu().numpy()
+        te = np.unique(idx)
+        n_touched.append(len(te))
+        touched_bytes.append(sum(expert_bytes(precs[e], cfg.H, cfg.I) for e in te))
+        pairs.append(idx.size)
+    io_bytes = cfg.T * (2 * cfg.H + 4 * cfg.E + 2 * cfg.H)
+
+    dist_barrier()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    t_step = time_graphs(step_graphs, steps, warmup, flush, stream)
+    clk = clocks.stop()
+    t_ffn = time_graphs(ffn_graphs, steps, warmup, flush, stream)
+    dist_barrier()
+
+    res = {"step_ms": float(np.mean(t_step)), "ffn_ms": float(np.mean(t_ffn)),
+           "step_ms_all": t_step, "clocks": clk,
+           "touched_bytes": float(np.mean([touched_bytes[i % n_batches] for i in range(steps)])),
+           "io_bytes": io_bytes, "n_touched": float(np.mean(n_touched)),
+           "pairs": float(np.mean(pairs)), "launches_per_step": 6}
+
+    if with_e2e:   # public API with host buffers: H2D inputs, forward, D2H output, every step
+        pin = [(lg.pin_memory(), x.pin_memory()) for lg, x in host_batches]
+        outs = [torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+                for _ in range(n_batches)]
+        dl = [torch.empty_like(d[0]) for d in dev_batches]
+        dx = [torch.empty_like(d[1]) for d in dev_batches]
+
+        def e2e_step(i):
+            b = i % n_batches
+            dl[b].copy_(pin[b][0], non_blocking=True)
+            dx[b].copy_(pin[b][1], non_blocking=True)
+            out = layer.forward(dl[b], dx[b], bufs=bufs[b], stream=stream)
+            outs[b].copy_(out, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for i in range(warmup):
+                e2e_step(i)
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps)]
+            for i in range(steps):
+                flush.zero_()
+                ev[i][0].record(stream)
+                e2e_step(i)
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+        res["e2e_ms"] = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+        res["h2d_bytes"] = pin[0][0].numel() * 4 + pin[0][1].numel() * 2
+        res["d2h_bytes"] = cfg.T * cfg.H * 2
+    status = B.moe_get_device_status()
+    if status:
+        raise RuntimeError(f"device status {status:#x} after the benchmark")
+    del step_graphs, ffn_graphs
+    layer.close()
+    return res
+
+
+class OracleRunner:
+    """The CPU oracle on the same workload (experts the batch selects only)."""
+
+    def __init__(self, cfg):
+        import oracle
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from helpers import oracle_experts
+        self.oracle, self.cfg = oracle, cfg
+        ranks = synth.zipf_ranks(cfg.E, cfg.seed)
+        precs = synth.precision_map(ranks, cfg.tiers)
+        self.logits = synth.gen_logits(cfg.T, cfg.E, cfg.seed * 1000, cfg.zipf_s, ranks)
+        self.x = synth.gen_x(cfg.T, cfg.H, cfg.seed * 1000)
+        idx = np.argsort(-self.logits, axis=1, kind="stable")[:, :cfg.k]
+        needed = set(np.unique(idx).tolist())
+        # unselected experts are never read; they stay in their bf16 master form
+        self.experts = oracle_experts(cfg.H, cfg.I, [precs[e] if e in needed else synth.BF16
+                                                     for e in range(cfg.E)], cfg.seed)
+        self.cores = oracle.num_threads()
+
+    def run(self, n_tok):
+        c = self.cfg
+        tokens = np.arange(min(n_tok, c.T), dtype=np.int32)
+        t0 = time.perf_counter()
+        self.oracle.moe_layer(self.logits, self.x, self.experts, c.k, c.H, c.I, tokens=tokens)
+        return len(tokens), time.perf_counter() - t0
+
+
+def oracle_baseline(cfg, budget_s=10.0):
+    """Time the CPU oracle on whole decode batches for about budget_s seconds."""
+    r = OracleRunner(cfg)
+    done, total = 0, 0.0
+    while total < budget_s:
+        n, dt = r.run(cfg.T)
+        done, total = done + n, total + dt
+    return {"value": done / total, "unit": "tokens/s", "cores": r.cores, "kind": "oracle",
+            "sample": f"{done // cfg.T} whole batches of {cfg.T} tokens of the {cfg.name} "
+                      f"workload ({total:.1f} s), binary64 C oracle"}
+
+
+# ----------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    cfg = synth.CONFIGS["qwen3_30b_decode"]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import oracle
+        oracle.build()
+        r = OracleRunner(cfg)
+        sample = 8   # tokens per step: a bounded slice of the 32-token batch
+        per = []
+        for i in range(args.warmup + args.steps):
+            n, dt = r.run(sample)
+            if i >= args.warmup:
+                per.append(dt / n)
+        v = 1.0 / float(np.mean(per))
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * sample * float(np.mean(per)), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": workload_name(cfg), "parallelism": "none (CPU)"},
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "kind": "oracle", "cores": r.cores,
+                                 "sample": f"{args.steps} steps of {sample} tokens of the "
+                                           f"{cfg.T}-token decode batch"},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    from mixed_precision_moe_b200 import build as mbuild
+    if rank == 0:
+        mbuild.build()
+    barrier()
+
+    hbm_gbs, tf_burst, tf_sust, peak_src = load_peaks()
+    dec = run_workload(cfg, args.steps, args.warmup, device, True, barrier)
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    step_ms = max_over_ranks(dec["step_ms"])
+    ffn_ms = max_over_ranks(dec["ffn_ms"])
+    e2e_ms = max_over_ranks(dec["e2e_ms"])
+    value = world * cfg.T / (step_ms * 1e-3)
+    ffn_gbs = dec["touched_bytes"] / (ffn_ms * 1e-3) / 1e9
+
+    prefill = None
+    if not args.no_prefill:
+        pcfg = synth.CONFIGS["qwen3_30b_prefill"]
+        pre = run_workload(pcfg, max(10, args.steps // 10), args.warmup, device, False, barrier)
+        p_step = max_over_ranks(pre["step_ms"])
+        p_ffn = max_over_ranks(pre["ffn_ms"])
+        flops = 6.0 * pcfg.H * pcfg.I * pre["pairs"]
+        tflops = flops / (p_ffn * 1e-3) / 1e12
+        prefill = {"workload": workload_name(pcfg), "value": world * pcfg.T / (p_step * 1e-3),
+                   "unit": "tokens/s", "ms_per_step": p_step, "ffn_ms": p_ffn,
+                   "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_burst,
+                                "unit": "TFLOP/s", "frac": tflops / tf_burst,
+                                "frac_of_spec_2250": tflops / 2250.0,
+                                "flops_per_launch": flops, "peak_source": peak_src + " burst",
+                                "traffic": None},
+                   "touched_experts": pre["n_touched"], "clocks": pre["clocks"]}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(cfg, budget_s=10.0)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; Qwen3-30B-A3B-shaped layer, random-init experts)",
+            "config": {"workload": workload_name(cfg), "global_batch": world * cfg.T,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed between steps (256 MiB write)", "graph": "CUDA graph per step"},
+            "roofline": {"bound": "hbm", "kernel": "grouped FFN (gate/up + down launches)",
+                         "achieved": ffn_gbs, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": ffn_gbs / hbm_gbs, "frac_of_8000": ffn_gbs / 8000.0,
+                         "bytes_per_launch": dec["touched_bytes"],
+                         "touched_experts": dec["n_touched"],
+                         "peak_source": peak_src, "traffic": None},
+            "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": dec["h2d_bytes"], "d2h_bytes_per_step": dec["d2h_bytes"]},
+            "gpu_launches": dec["launches_per_step"] * args.steps,
+            "clocks": dec["clocks"],
+            "cpu_baseline": cpu,
+            "prefill": prefill,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,405 @@
+// moe_lib.cu -- host side of the libmoe C ABI (include/moe.h) and the single
+// translation unit that holds every kernel of the library.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "grouped_ffn.cuh"
+#include "route_permute_combine.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+#define MOE_CUDA_TRY(expr)                                                              \
+  do {                                                                                  \
+    cudaError_t err_ = (expr);                                                          \
+    if (err_ != cudaSuccess)                                                            \
+      return fail(MOE_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(err_));      \
+  } while (0)
+
+#define MOE_CHECK(cond, code, ...) \
+  do {                             \
+    if (!(cond)) return fail(code, __VA_ARGS__); \
+  } while (0)
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [rows][cols] matrix of `esize`-byte elements,
+// box = box_rows x box_cols elements.
+int encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int esize,
+              uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+              CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  MOE_CHECK(fn != nullptr, MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)esize};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MOE_CHECK(r == CUDA_SUCCESS, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOE_OK;
+}
+
+// Tensor map of one expert weight matrix [rows][K] in its storage format:
+// BF16 -> box 128 rows x 64 bf16 (128-byte swizzle, the MMA operand layout);
+// INT8/INT4 -> box 128 rows x 64 bytes of codes (staged, then dequantised).
+int encode_weight(CUtensorMap* m, const void* base, int prec, int rows, int K) {
+  if (prec == MOE_BF16)
+    return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 128, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  const int cols = (prec == MOE_INT4) ? K / 2 : K;
+  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, 128, 64,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+int num_sms(int device) {
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return 0;
+  return n;
+}
+
+}  // namespace
+
+struct moe_layer {
+  int H, I, E, k;
+  int device;
+  moe::ffn::ExpertDesc* d_descs;  // [E], device
+  std::vector<int> prec;          // host shadow, -1 = unset
+};
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+int moe_abi_version(void) { return 1; }
+
+int moe_layer_create(int H, int I, int E, int k, moe_layer_t* out) {
+  MOE_CHECK(out != nullptr, MOE_ERR_INVALID_ARG, "out is null");
+  *out = nullptr;
+  MOE_CHECK(H > 0 && I > 0 && H % 128 == 0 && I % 128 == 0, MOE_ERR_UNSUPPORTED,
+            "H=%d and I=%d must be positive multiples of 128", H, I);
+  MOE_CHECK(E >= 1 && E <= moe::ffn::kMaxE, MOE_ERR_UNSUPPORTED, "E=%d outside [1, 512]", E);
+  MOE_CHECK(k >= 1 && k <= 16 && k <= E, MOE_ERR_INVALID_ARG, "k=%d outside [1, min(E, 16)]", k);
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  moe::ffn::ExpertDesc* d = nullptr;
+  MOE_CUDA_TRY(cudaMalloc(&d, sizeof(moe::ffn::ExpertDesc) * E));
+  // All bytes 0xFF: prec = -1 (unset) for every expert.
+  cudaError_t e1 = cudaMemset(d, 0xFF, sizeof(moe::ffn::ExpertDesc) * E);
+  cudaError_t e2 = cudaDeviceSynchronize();
+  if (e1 != cudaSuccess || e2 != cudaSuccess) {
+    cudaFree(d);
+    return fail(MOE_ERR_CUDA, "descriptor table init failed: %s",
+                cudaGetErrorString(e1 != cudaSuccess ? e1 : e2));
+  }
+  moe_layer* L = new moe_layer{H, I, E, k, dev, d, std::vector<int>(E, -1)};
+  *out = L;
+  return ok();
+}
+
+int moe_layer_destroy(moe_layer_t layer) {
+  MOE_CHECK(layer != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  cudaDeviceSynchronize();
+  cudaError_t e = cudaFree(layer->d_descs);
+  delete layer;
+  MOE_CHECK(e == cudaSuccess, MOE_ERR_CUDA, "cudaFree failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+int moe_set_expert_precision(moe_layer_t L, int expert, moe_precision_t precision,
+                             const moe_expert_weights* w, void* stream) {
+  MOE_CHECK(L != nullptr && w != nullptr, MOE_ERR_INVALID_ARG, "null layer or weights");
+  MOE_CHECK(expert >= 0 && expert < L->E, MOE_ERR_INVALID_ARG, "expert %d outside [0, %d)",
+            expert, L->E);
+  const int prec = (int)precision;
+  MOE_CHECK(prec == MOE_BF16 || prec == MOE_INT8 || prec == MOE_INT4, MOE_ERR_INVALID_ARG,
+            "unknown precision %d", prec);
+  MOE_CHECK(w->w13 != nullptr && w->w2 != nullptr, MOE_ERR_INVALID_ARG, "null weight pointer");
+  MOE_CHECK(aligned(w->w13, 16) && aligned(w->w2, 16), MOE_ERR_UNSUPPORTED,
+            "weight buffers must be 16-byte aligned");
+  if (prec != MOE_BF16) {
+    MOE_CHECK(w->s13 != nullptr && w->s2 != nullptr, MOE_ERR_INVALID_ARG,
+              "INT8/INT4 experts need scales");
+    MOE_CHECK(aligned(w->s13, 16) && aligned(w->s2, 16), MOE_ERR_UNSUPPORTED,
+              "scale buffers must be 16-byte aligned");
+  }
+  moe::ffn::ExpertDesc d;
+  memset(&d, 0, sizeof d);
+  int rc = encode_weight(&d.tm_w13, w->w13, prec, 2 * L->I, L->H);
+  if (rc != MOE_OK) return rc;
+  rc = encode_weight(&d.tm_w2, w->w2, prec, L->H, L->I);
+  if (rc != MOE_OK) return rc;
+  d.s13 = prec == MOE_BF16 ? nullptr : static_cast<const __half*>(w->s13);
+  d.s2 = prec == MOE_BF16 ? nullptr : static_cast<const __half*>(w->s2);
+  d.prec = prec;
+  moe::ffn::write_desc_kernel<<<1, 32, 0, as_stream(stream)>>>(L->d_descs + expert, d);
+  MOE_CUDA_TRY(cudaGetLastError());
+  L->prec[expert] = prec;
+  return ok();
+}
+
+int moe_get_expert_precision(moe_layer_t L, int expert, int* precision) {
+  MOE_CHECK(L != nullptr && precision != nullptr, MOE_ERR_INVALID_ARG, "null argument");
+  MOE_CHECK(expert >= 0 && expert < L->E, MOE_ERR_INVALID_ARG, "expert %d outside [0, %d)",
+            expert, L->E);
+  *precision = L->prec[expert];
+  return ok();
+}
+
+int moe_route_topk(const float* logits, int T, int E, int k, int renormalize, int32_t* topk_idx,
+                   float* topk_w, void* stream) {
+  MOE_CHECK(T >= 0, MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  MOE_CHECK(E >= 1 && E <= 512, MOE_ERR_UNSUPPORTED, "E=%d outside [1, 512]", E);
+  MOE_CHECK(k >= 1 && k <= 16 && k <= E, MOE_ERR_INVALID_ARG, "k=%d outside [1, min(E, 16)]", k);
+  if (T == 0) return ok();
+  MOE_CHECK(logits && topk_idx && topk_w, MOE_ERR_INVALID_ARG, "null pointer");
+  const int keys = (E + 31) / 32;
+  const dim3 block(256), grid((T + 7) / 8);
+  cudaStream_t s = as_stream(stream);
+  if (keys <= 1)
+    moe::route_topk_kernel<1><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
+  else if (keys <= 2)
+    moe::route_topk_kernel<2><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
+  else if (keys <= 4)
+    moe::route_topk_kernel<4><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
+  else if (keys <= 8)
+    moe::route_topk_kernel<8><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
+  else
+    moe::route_topk_kernel<16><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
+  MOE_CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int H,
+                int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row, void* x_perm,
+                void* stream) {
+  MOE_CHECK(T >= 0, MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  MOE_CHECK(E >= 1 && E <= 512, MOE_ERR_UNSUPPORTED, "E=%d outside [1, 512]", E);
+  MOE_CHECK(k >= 1 && k <= 16, MOE_ERR_INVALID_ARG, "k=%d outside [1, 16]", k);
+  MOE_CHECK(H > 0 && H % 8 == 0, MOE_ERR_UNSUPPORTED, "H=%d must be a positive multiple of 8", H);
+  MOE_CHECK(expert_offsets != nullptr, MOE_ERR_INVALID_ARG, "null expert_offsets");
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {
+    MOE_CUDA_TRY(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), s));
+    return ok();
+  }
+  MOE_CHECK(topk_idx && x && perm_token && dest_row && x_perm, MOE_ERR_INVALID_ARG,
+            "null pointer");
+  MOE_CHECK(aligned(x, 16) && aligned(x_perm, 16), MOE_ERR_UNSUPPORTED,
+            "x and x_perm must be 16-byte aligned");
+  const size_t smem = moe::permute_smem_bytes(E);
+  static bool attr_set = false;
+  if (!attr_set) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(moe::permute_index_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)moe::permute_smem_bytes(512)));
+    attr_set = true;
+  }
+  moe::permute_index_kernel<<<1, moe::kPermuteThreads, smem, s>>>(topk_idx, T, E, k, expert_offsets,
+                                                                  perm_token, dest_row);
+  MOE_CUDA_TRY(cudaGetLastError());
+  const int vec = H / 8;
+  const long long nvec = (long long)T * k * vec;
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  const long long cap = (long long)num_sms(dev) * 8;
+  const int blocks = (int)std::max(1LL, std::min(cap, (nvec + 255) / 256));
+  moe::gather_rows_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), perm_token,
+                                                  expert_offsets, E, vec,
+                                                  static_cast<uint4*>(x_perm));
+  MOE_CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+int moe_ffn_workspace_bytes(moe_layer_t L, int rows, size_t* bytes) {
+  MOE_CHECK(L != nullptr && bytes != nullptr, MOE_ERR_INVALID_ARG, "null argument");
+  MOE_CHECK(rows >= 0, MOE_ERR_INVALID_ARG, "rows=%d < 0", rows);
+  const size_t h = ((size_t)rows * L->I * 2 + 255) / 256 * 256;
+  *bytes = h + 256;  // h [rows][I] bf16, then the scheduler's counters
+  return ok();
+}
+
+int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expert_offsets,
+                          int rows, void* y_perm, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  using namespace moe::ffn;
+  MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  MOE_CHECK(rows >= 0, MOE_ERR_INVALID_ARG, "rows=%d < 0", rows);
+  if (rows == 0) return ok();
+  MOE_CHECK(x_perm && expert_offsets && y_perm && workspace, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_CHECK(aligned(x_perm, 16) && aligned(y_perm, 16), MOE_ERR_UNSUPPORTED,
+            "x_perm and y_perm must be 16-byte aligned");
+  MOE_CHECK(aligned(workspace, 256), MOE_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+  size_t need = 0;
+  moe_ffn_workspace_bytes(L, rows, &need);
+  MOE_CHECK(workspace_bytes >= need, MOE_ERR_INVALID_ARG, "workspace %zu B < %zu B needed",
+            workspace_bytes, need);
+  for (int e = 0; e < L->E; ++e)
+    MOE_CHECK(L->prec[e] >= 0, MOE_ERR_NOT_MATERIALIZED, "expert %d has no weights", e);
+
+  cudaStream_t s = as_stream(stream);
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  const int grid = num_sms(dev);
+  MOE_CHECK(grid > 0, MOE_ERR_CUDA, "cannot query the SM count");
+
+  auto* h = static_cast<__nv_bfloat16*>(workspace);
+  int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + need - 256);
+  MOE_CUDA_TRY(cudaMemsetAsync(counters, 0, 2 * sizeof(int), s));
+
+  // Every expert holds at most T = rows / k rows; up to 128 rows fit one swap-mode tile.
+  const int T = (rows + L->k - 1) / L->k;
+  const bool swap = T <= 128;
+  const int xbox = swap ? 16 : 128;
+
+  CUtensorMap tm_x, tm_h;
+  int rc = encode_2d(&tm_x, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->H, xbox, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != MOE_OK) return rc;
+  rc = encode_2d(&tm_h, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->I, xbox, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != MOE_OK) return rc;
+
+  Params pg{L->d_descs, expert_offsets, h, counters, L->E, L->H, L->I, L->H, L->I, L->I / 128, xbox};
+  Params pd{L->d_descs, expert_offsets, static_cast<__nv_bfloat16*>(y_perm), counters + 1, L->E,
+            L->H, L->I, L->I, L->H, (L->H + 255) / 256, xbox};
+
+  static bool attr_set = false;
+  const int smem = (int)smem_bytes();
+  if (!attr_set) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<true, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<false, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<true, false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<false, false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr_set = true;
+  }
+  if (swap) {
+    grouped_ffn_kernel<true, true><<<grid, kThreads, smem, s>>>(tm_x, pg);
+    MOE_CUDA_TRY(cudaGetLastError());
+    grouped_ffn_kernel<false, true><<<grid, kThreads, smem, s>>>(tm_h, pd);
+  } else {
+    grouped_ffn_kernel<true, false><<<grid, kThreads, smem, s>>>(tm_x, pg);
+    MOE_CUDA_TRY(cudaGetLastError());
+    grouped_ffn_kernel<false, false><<<grid, kThreads, smem, s>>>(tm_h, pd);
+  }
+  MOE_CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w, int T, int k,
+                int H, void* out, void* stream) {
+  MOE_CHECK(T >= 0, MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  MOE_CHECK(k >= 1 && k <= 16, MOE_ERR_INVALID_ARG, "k=%d outside [1, 16]", k);
+  MOE_CHECK(H > 0 && H % 8 == 0, MOE_ERR_UNSUPPORTED, "H=%d must be a positive multiple of 8", H);
+  if (T == 0) return ok();
+  MOE_CHECK(y_perm && dest_row && topk_w && out, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_CHECK(aligned(y_perm, 16) && aligned(out, 16), MOE_ERR_UNSUPPORTED,
+            "y_perm and out must be 16-byte aligned");
+  const int vec = H / 8;
+  const dim3 block(std::min(256, ((vec + 31) / 32) * 32));
+  const dim3 grid(T, (vec + block.x - 1) / block.x);
+  moe::combine_kernel<<<grid, block, 0, as_stream(stream)>>>(
+      static_cast<const uint4*>(y_perm), dest_row, topk_w, k, vec, static_cast<uint4*>(out));
+  MOE_CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, int renormalize,
+                      int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                      int32_t* perm_token, int32_t* dest_row, void* x_perm, void* y_perm,
+                      void* workspace, size_t workspace_bytes, void* out, void* stream) {
+  MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  int rc = moe_route_topk(logits, T, L->E, L->k, renormalize, topk_idx, topk_w, stream);
+  if (rc != MOE_OK) return rc;
+  rc = moe_permute(topk_idx, x, T, L->E, L->k, L->H, expert_offsets, perm_token, dest_row, x_perm,
+                   stream);
+  if (rc != MOE_OK) return rc;
+  rc = moe_grouped_ffn_mixed(L, x_perm, expert_offsets, T * L->k, y_perm, workspace,
+                             workspace_bytes, stream);
+  if (rc != MOE_OK) return rc;
+  return moe_combine(y_perm, dest_row, topk_w, T, L->k, L->H, out, stream);
+}
+
+int moe_quantize_weights(const void* w_bf16, int rows, int K, moe_precision_t precision,
+                         void* q_out, void* scales, void* stream) {
+  const int prec = (int)precision;
+  MOE_CHECK(prec == MOE_INT8 || prec == MOE_INT4, MOE_ERR_INVALID_ARG,
+            "quantiser precision must be INT8 or INT4");
+  MOE_CHECK(rows >= 0 && K > 0 && K % 128 == 0, MOE_ERR_UNSUPPORTED,
+            "rows=%d, K=%d (K must be a positive multiple of 128)", rows, K);
+  if (rows == 0) return ok();
+  MOE_CHECK(w_bf16 && q_out && scales, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_CHECK(aligned(w_bf16, 8) && aligned(q_out, 4) && aligned(scales, 2), MOE_ERR_UNSUPPORTED,
+            "misaligned buffer");
+  const long long warps = (long long)rows * (K / 128);
+  const long long blocks = (warps * 32 + 255) / 256;
+  MOE_CHECK(blocks < (1LL << 31), MOE_ERR_UNSUPPORTED, "matrix too large");
+  moe::quantize_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(
+      static_cast<const uint16_t*>(w_bf16), rows, K, prec, static_cast<uint8_t*>(q_out),
+      static_cast<uint16_t*>(scales));
+  MOE_CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+int moe_get_device_status(unsigned int* status) {
+  MOE_CHECK(status != nullptr, MOE_ERR_INVALID_ARG, "status is null");
+  MOE_CUDA_TRY(cudaDeviceSynchronize());
+  unsigned int v = 0, zero = 0;
+  MOE_CUDA_TRY(cudaMemcpyFromSymbol(&v, moe::g_status, sizeof v));
+  MOE_CUDA_TRY(cudaMemcpyToSymbol(moe::g_status, &zero, sizeof zero));
+  *status = v;
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,336 @@
+// route_permute_combine.cuh -- the memory-light steps of the routed-expert
+// layer: top-k routing, grouping by expert, weighted combine, and the
+// group-128 quantiser used to build INT8/INT4 experts.
+//
+// All follow "Every Expert Counts: ExactMoE for Memory-Efficient W4A16
+// Inference": routing equation of Section 3.1, grouping of Figure 1, combine of
+// Section 3.4, quantiser equation of Section 3.2.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------------ routing --
+
+// Orderable key of a logit: larger key <=> larger value, -0.0 and +0.0 share a
+// key, NaN takes the key of -inf.  Every real key is >= 0x007FFFFF, so 0 marks
+// an empty slot.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  uint32_t u = __float_as_uint(v);
+  if ((u << 1) == 0) u = 0;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// One warp per token.  Lane l holds the keys of experts l, l+32, ... (KEYS
+// slots, ascending id).  k rounds of warp argmax pick the experts by
+// descending logit, ties to the lowest id; lane j keeps the j-th pick.
+template <int KEYS>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
+                                                         int E, int k, int renormalize,
+                                                         int32_t* __restrict__ topk_idx,
+                                                         float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* z = logits + (size_t)t * E;
+
+  uint32_t key[KEYS];
+  bool nan_seen = false;
+#pragma unroll
+  for (int i = 0; i < KEYS; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = 0;
+    if (e < E) {
+      float v = z[e];
+      if (isnan(v)) {
+        nan_seen = true;
+        v = -INFINITY;
+      }
+      key[i] = logit_key(v);
+    }
+  }
+  if (__any_sync(0xffffffffu, nan_seen) && lane == 0) flag_status(MOE_STATUS_NONFINITE_LOGIT);
+
+  int my_e = 0;
+  float my_z = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    uint32_t best = 0;
+    int best_i = -1;
+#pragma unroll
+    for (int i = 0; i < KEYS; ++i)
+      if (key[i] > best) {  // strict: the lowest id among this lane's equal keys
+        best = key[i];
+        best_i = i;
+      }
+    const uint32_t win_key = __reduce_max_sync(0xffffffffu, best);
+    const uint32_t cand =
+        (best_i >= 0 && best == win_key) ? (uint32_t)(lane + 32 * best_i) : 0xffffffffu;
+    const uint32_t win_e = __reduce_min_sync(0xffffffffu, cand);
+    if ((int)(win_e & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < KEYS; ++i)
+        if (i == (int)(win_e >> 5)) key[i] = 0;
+    }
+    if (lane == j) {
+      my_e = (int)win_e;
+      my_z = key_logit(win_key);
+    }
+  }
+
+  // Gating weights.  m = the largest selected logit (pick 0).
+  const float m = __shfl_sync(0xffffffffu, my_z, 0);
+  const float ex = (lane < k) ? expf(my_z - m) : 0.0f;
+  float den = 0.0f;
+  if (renormalize) {
+    for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, ex, j);
+  } else {
+    float part = 0.0f;
+    for (int e = lane; e < E; e += 32) {
+      const float v = z[e];
+      if (!isnan(v)) part += expf(v - m);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    den = part;
+  }
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = my_e;
+    topk_w[(size_t)t * k + lane] = ex / den;
+  }
+}
+
+// -------------------------------------------------------------- permutation --
+
+constexpr int kPermuteThreads = 1024;
+constexpr int kPermuteWarps = kPermuteThreads / 32;
+
+__host__ __device__ constexpr size_t permute_smem_bytes(int E) {
+  return (size_t)(2 * kPermuteWarps + 1) * E * sizeof(int32_t);
+}
+
+// Whole grouping in one CTA.  Warp w owns a contiguous chunk of tokens.
+//   1. per-(warp, expert) counts (shared-memory atomics: order-free sums)
+//   2. exclusive scan over (expert, warp) -> expert_offsets and per-warp bases
+//   3. each warp walks its tokens 32 at a time in token order; a token's rank
+//      inside expert e is the number of lower lanes that also chose e, read
+//      from a per-(warp, expert) lane bitmask.
+// The resulting order (expert id, then token) is fixed; no atomic decides it.
+__global__ void __launch_bounds__(kPermuteThreads, 1)
+    permute_index_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                         int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+                         int32_t* __restrict__ dest_row) {
+  extern __shared__ int32_t psm[];
+  int32_t* base = psm;                                          // [warps][E]
+  uint32_t* mask = reinterpret_cast<uint32_t*>(psm + kPermuteWarps * E);  // [warps][E]
+  int32_t* tot = psm + 2 * kPermuteWarps * E;                   // [E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int i = tid; i < 2 * kPermuteWarps * E; i += blockDim.x) psm[i] = 0;
+  __syncthreads();
+
+  const int chunk = (T + kPermuteWarps - 1) / kPermuteWarps;
+  const int t_begin = min(T, warp * chunk);
+  const int t_end = min(T, t_begin + chunk);
+
+  // 1. counts of the valid pairs
+  bool bad = false;
+  for (int t = t_begin + lane; t < t_end; t += 32) {
+    int ev[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) ev[j] = (j < k) ? idx[(size_t)t * k + j] : -1;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j >= k) break;
+      bool ok = ev[j] >= 0 && ev[j] < E;
+#pragma unroll
+      for (int jj = 0; jj < j; ++jj) ok = ok && (ev[jj] != ev[j]);
+      if (ok)
+        atomicAdd(&base[warp * E + ev[j]], 1);
+      else
+        bad = true;
+    }
+  }
+  if (bad) flag_status(MOE_STATUS_BAD_EXPERT_ID);
+  __syncthreads();
+
+  // 2a. per expert, exclusive prefix over warps
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < kPermuteWarps; ++w) {
+      const int c = base[w * E + e];
+      base[w * E + e] = run;
+      run += c;
+    }
+    tot[e] = run;
+  }
+  __syncthreads();
+  // 2b. exclusive scan of the expert totals (warp 0; lane owns a run of ids)
+  if (warp == 0) {
+    const int per = (E + 31) / 32;
+    const int e0 = lane * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i)
+      if (e0 + i < E) local += tot[e0 + i];
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    int run = incl - local;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < E) {
+        const int c = tot[e];
+        tot[e] = run;
+        offsets[e] = run;
+        run += c;
+      }
+    }
+    if (lane == 31) offsets[E] = incl;
+  }
+  __syncthreads();
+  for (int i = tid; i < kPermuteWarps * E; i += blockDim.x) base[i] += tot[i % E];
+  __syncthreads();
+
+  // 3. stable scatter
+  int32_t* wbase = base + warp * E;
+  uint32_t* wmask = mask + warp * E;
+  const uint32_t lower = (1u << lane) - 1u;
+  for (int tb = t_begin; tb < t_end; tb += 32) {
+    const int t = tb + lane;
+    const bool tv = t < t_end;
+    int ev[16];
+    bool ok[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      ev[j] = (tv && j < k) ? idx[(size_t)t * k + j] : -1;
+      ok[j] = ev[j] >= 0 && ev[j] < E;
+#pragma unroll
+      for (int jj = 0; jj < j; ++jj) ok[j] = ok[j] && (ev[jj] != ev[j]);
+      if (ok[j]) atomicOr(&wmask[ev[j]], 1u << lane);
+    }
+    __syncwarp();
+    uint32_t mm[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      mm[j] = 0;
+      if (ok[j]) {
+        mm[j] = wmask[ev[j]];
+        const int row = wbase[ev[j]] + __popc(mm[j] & lower);
+        dest_row[(size_t)t * k + j] = row;
+        perm_token[row] = t;
+      } else if (tv && j < k) {
+        dest_row[(size_t)t * k + j] = -1;
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (ok[j] && (mm[j] & lower) == 0) {  // lowest lane of this expert updates
+        wbase[ev[j]] += __popc(mm[j]);
+        wmask[ev[j]] = 0;
+      }
+    __syncwarp();
+  }
+}
+
+// x_perm[r] = x[perm_token[r]] for r < offsets[E], 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                          const int32_t* __restrict__ perm_token,
+                                                          const int32_t* __restrict__ offsets,
+                                                          int E, int vec_per_row,
+                                                          uint4* __restrict__ x_perm) {
+  const size_t n = (size_t)offsets[E] * vec_per_row;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = i / vec_per_row, c = i % vec_per_row;
+    x_perm[i] = x[(size_t)perm_token[r] * vec_per_row + c];
+  }
+}
+
+// ------------------------------------------------------------------ combine --
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// out[t] = sum_j w[t][j] * y[dest_row[t][j]] in fp32, j = 0..k-1 in order.
+// grid (T, ceil(H/8 / blockDim.x)); each thread one 16-byte vector of a row.
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y,
+                                                      const int32_t* __restrict__ dest_row,
+                                                      const float* __restrict__ topk_w, int k,
+                                                      int vec_per_row, uint4* __restrict__ out) {
+  const int t = blockIdx.x;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;
+  if (c >= vec_per_row) return;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int j = 0; j < k; ++j) {
+    const int r = dest_row[(size_t)t * k + j];
+    if (r < 0) continue;
+    const float wj = topk_w[(size_t)t * k + j];
+    float f[8];
+    bf16x8_to_f32(y[(size_t)r * vec_per_row + c], f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+  }
+  uint4 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  o.z = pack_bf16x2(acc[4], acc[5]);
+  o.w = pack_bf16x2(acc[6], acc[7]);
+  out[(size_t)t * vec_per_row + c] = o;
+}
+
+// ---------------------------------------------------------------- quantiser --
+
+// One warp per (row, K-group of 128); lane holds 4 consecutive elements.
+// s = fp16_rne(amax / Q) (binary32 quotient), q = clip(rint_even(W / s)).
+__global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restrict__ w, int rows,
+                                                       int K, int prec, uint8_t* __restrict__ q,
+                                                       uint16_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int groups = K / 128;
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (gw >= (long long)rows * groups) return;
+  const int row = (int)(gw / groups), g = (int)(gw % groups);
+  const uint2 raw = *reinterpret_cast<const uint2*>(w + (size_t)row * K + g * 128 + lane * 4);
+  float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+  uint32_t amax_bits = 0;  // |v| as non-negative float bits order like the values
+#pragma unroll
+  for (int i = 0; i < 4; ++i) amax_bits = max(amax_bits, __float_as_uint(fabsf(v[i])));
+  amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
+  const int Q = (prec == MOE_INT4) ? 7 : 127;
+  const __half sh = __float2half_rn(__fdiv_rn(__uint_as_float(amax_bits), (float)Q));
+  const float s = __half2float(sh);
+  int qv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int c = 0;
+    if (s != 0.0f) c = __float2int_rn(__fdiv_rn(v[i], s));
+    qv[i] = min(Q, max(-Q - 1, c));
+  }
+  if (lane == 0) scales[(size_t)g * rows + row] = __half_as_ushort(sh);
+  if (prec == MOE_INT8) {
+    const uint32_t packed = (uint32_t)(qv[0] & 0xFF) | ((uint32_t)(qv[1] & 0xFF) << 8) |
+                            ((uint32_t)(qv[2] & 0xFF) << 16) | ((uint32_t)(qv[3] & 0xFF) << 24);
+    *reinterpret_cast<uint32_t*>(q + (size_t)row * K + g * 128 + lane * 4) = packed;
+  } else {
+    const uint16_t packed = (uint16_t)((qv[0] + 8) | ((qv[1] + 8) << 4) | ((qv[2] + 8) << 8) |
+                                       ((qv[3] + 8) << 12));
+    *reinterpret_cast<uint16_t*>(q + (size_t)row * (K / 2) + g * 64 + lane * 2) = packed;
+  }
+}
+
+}  // namespace moe

@@ -162,6 +162,7 @@ int oracle_quantize(const uint16_t* w, int rows, int K, int prec, void* q_out,
   const int Q = (prec == OR_INT4) ? 7 : 127;
   const int qmin = -(Q + 1), qmax = Q;
   if (prec == OR_INT4) memset(q_out, 0, (size_t)rows * (K / 2));
+#pragma omp parallel for schedule(static)
   for (int r = 0; r < rows; ++r) {
     for (int g = 0; g < K / 128; ++g) {
       float amax = 0.0f;
@@ -249,10 +250,20 @@ int oracle_route_topk(const float* logits, int T, int E, int k, int renormalize,
 /* Permutation (Figure 1: tokens grouped by selected expert)                 */
 /* ------------------------------------------------------------------------ */
 
+/* A pair is invalid when its id lies outside [0, E) or repeats an id of an
+ * earlier slot of the same token (a top-k set has distinct members). */
+static int pair_invalid(const int32_t* idx, int E, int k, int t, int j) {
+  int e = idx[(size_t)t * k + j];
+  if (e < 0 || e >= E) return 1;
+  for (int jj = 0; jj < j; ++jj)
+    if (idx[(size_t)t * k + jj] == e) return 1;
+  return 0;
+}
+
 /* Counting sort of the (token, slot) pairs by expert, stable by token.
  * offsets [E+1], perm_token [rows] (row -> token), dest_row [T*k]
- * (pair -> row, -1 for a pair whose id lies outside [0, E)).
- * Returns the number of such invalid pairs (0 for valid input). */
+ * (pair -> row, -1 for an invalid pair).
+ * Returns the number of invalid pairs (0 for valid input). */
 int oracle_permute(const int32_t* idx, int T, int E, int k, int32_t* offsets,
                    int32_t* perm_token, int32_t* dest_row) {
   if (T < 0 || E <= 0 || k <= 0) return OR_ERR_ARG;
@@ -260,18 +271,16 @@ int oracle_permute(const int32_t* idx, int T, int E, int k, int32_t* offsets,
   if (!cursor) return OR_ERR_NOMEM;
   int invalid = 0;
   for (int e = 0; e <= E; ++e) offsets[e] = 0;
-  for (size_t p = 0; p < (size_t)T * k; ++p) {
-    int e = idx[p];
-    if (e < 0 || e >= E) continue;
-    offsets[e + 1] += 1;
-  }
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j)
+      if (!pair_invalid(idx, E, k, t, j)) offsets[idx[(size_t)t * k + j] + 1] += 1;
   for (int e = 0; e < E; ++e) offsets[e + 1] += offsets[e];
   for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
   for (int t = 0; t < T; ++t) {
     for (int j = 0; j < k; ++j) {
       size_t p = (size_t)t * k + j;
       int e = idx[p];
-      if (e < 0 || e >= E) {
+      if (pair_invalid(idx, E, k, t, j)) {
         dest_row[p] = -1;
         invalid += 1;
         continue;

@@ -146,10 +146,11 @@ def test_permute_invariants_and_bruteforce():
 
 
 def test_permute_marks_invalid_ids():
-    idx = np.array([[0, 5], [-1, 1]], np.int32)
+    idx = np.array([[0, 5], [-1, 1], [1, 1]], np.int32)
     off, perm_token, dest, inv = oracle.permute(idx, 2)
-    assert inv == 2 and list(off) == [0, 1, 2]
-    assert dest[0, 1] == -1 and dest[1, 0] == -1
+    assert inv == 3 and list(off) == [0, 1, 3]
+    assert dest[0, 1] == -1 and dest[1, 0] == -1 and dest[2, 1] == -1
+    assert list(perm_token[:3]) == [0, 1, 2] and list(dest[:, 0]) == [0, -1, 2]
 
 
 # ------------------------------------------------------------- quantiser --
