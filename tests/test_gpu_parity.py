@@ -166,6 +166,17 @@ def test_combine_matches_oracle_and_skips_missing_pairs():
 FFN_GROUPS = [1, 3, 16, 17, 64, 127, 128, 129, 200, 256, 0, 300]
 
 
+def _mode_k(mode, groups):
+    """The library picks the MMA orientation from T = ceil(rows / k): weights-as-M
+    ("swap") when T <= 128, tokens-as-M ("tile") otherwise."""
+    R, E = sum(groups), len(groups)
+    if mode == "swap":
+        assert -(-R // E) <= 128
+        return E
+    assert R > 128
+    return 1
+
+
 def _ffn_case(H, I, precs, groups, seed, random_codes=False):
     E = len(groups)
     exps = oracle_experts(H, I, precs, seed)
@@ -181,13 +192,13 @@ def _ffn_case(H, I, precs, groups, seed, random_codes=False):
     return exps, offsets, x_perm, y_o
 
 
-@pytest.mark.parametrize("mode_k", [16, 1], ids=["swap", "tile"])
+@pytest.mark.parametrize("mode", ["swap", "tile"])
 @pytest.mark.parametrize("H,I", [(512, 384), (384, 256)])
-def test_grouped_ffn_mixed_precisions_ragged_groups(mode_k, H, I):
+def test_grouped_ffn_mixed_precisions_ragged_groups(mode, H, I):
     precs = [oracle.BF16, oracle.INT8, oracle.INT4] * 4
     exps, offsets, x_perm, y_o = _ffn_case(H, I, precs, FFN_GROUPS, 50 + H)
     E = len(FFN_GROUPS)
-    layer = gpu_layer(H, I, E, mode_k, exps)
+    layer = gpu_layer(H, I, E, _mode_k(mode, FFN_GROUPS), exps)
     y = B.moe_grouped_ffn_mixed(layer, to_gpu_bf16(x_perm), torch.from_numpy(offsets).cuda())
     y = bf16_to_f64(y)
     for e in range(E):
@@ -199,26 +210,26 @@ def test_grouped_ffn_mixed_precisions_ragged_groups(mode_k, H, I):
     layer.close()
 
 
-@pytest.mark.parametrize("mode_k", [16, 1], ids=["swap", "tile"])
-def test_grouped_ffn_arbitrary_codes(mode_k):
+@pytest.mark.parametrize("mode", ["swap", "tile"])
+def test_grouped_ffn_arbitrary_codes(mode):
     H, I = 256, 256
     groups = [5, 128, 33, 0, 77, 1]
     precs = [oracle.INT4, oracle.INT8, oracle.INT4, oracle.INT8, oracle.INT8, oracle.INT4]
     exps, offsets, x_perm, y_o = _ffn_case(H, I, precs, groups, 77, random_codes=True)
-    layer = gpu_layer(H, I, len(groups), mode_k, exps)
+    layer = gpu_layer(H, I, len(groups), _mode_k(mode, groups), exps)
     y = B.moe_grouped_ffn_mixed(layer, to_gpu_bf16(x_perm), torch.from_numpy(offsets).cuda())
     check_close(bf16_to_f64(y), y_o, "arbitrary codes")
     layer.close()
 
 
-@pytest.mark.parametrize("mode_k", [16, 1], ids=["swap", "tile"])
-def test_grouped_equals_per_expert_launch_bit_for_bit(mode_k):
+@pytest.mark.parametrize("mode", ["swap", "tile"])
+def test_grouped_equals_per_expert_launch_bit_for_bit(mode):
     H, I = 256, 256
     groups = [40, 0, 129, 7, 64]
     precs = [oracle.INT4, oracle.BF16, oracle.INT8, oracle.BF16, oracle.INT4]
     exps, offsets, x_perm, _ = _ffn_case(H, I, precs, groups, 91)
     E = len(groups)
-    layer = gpu_layer(H, I, E, mode_k, exps)
+    layer = gpu_layer(H, I, E, _mode_k(mode, groups), exps)
     xg = to_gpu_bf16(x_perm)
     y1 = B.moe_grouped_ffn_mixed(layer, xg, torch.from_numpy(offsets).cuda())
     y2 = B.moe_grouped_ffn_mixed(layer, xg, torch.from_numpy(offsets).cuda())
@@ -328,9 +339,11 @@ def test_wave_split_sums_to_whole_layer():
     wave = idx < cfg.E // 2          # experts 0..3 in wave A, 4..7 in wave B
     neg = torch.full_like(dest, -1)
     whole = bf16_to_f64(B.moe_combine(y, dest, w))
-    part = (bf16_to_f64(B.moe_combine(y, torch.where(wave, dest, neg), w)) +
-            bf16_to_f64(B.moe_combine(y, torch.where(wave, neg, dest), w)))
-    assert np.all(np.abs(part - whole) <= 2.0 ** -7 * np.abs(whole) + 1e-6)
+    a = bf16_to_f64(B.moe_combine(y, torch.where(wave, dest, neg), w))
+    b = bf16_to_f64(B.moe_combine(y, torch.where(wave, neg, dest), w))
+    # each of a, b, whole carries one bf16 rounding (<= 2^-9 relative to itself)
+    # on top of an fp32 sum; the partial sums may be larger than their total
+    assert np.all(np.abs(a + b - whole) <= 2.0 ** -8 * (np.abs(a) + np.abs(b) + np.abs(whole)) + 1e-6)
     layer.close()
 
 
