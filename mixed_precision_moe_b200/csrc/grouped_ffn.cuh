@@ -7,33 +7,35 @@
 // fused gate/up projection and one down projection" per group of experts).
 // Experts in one launch may be BF16, INT8 or INT4 (MxMoE abstract: GEMMs of
 // different precisions in one grouped kernel); INT8/INT4 weights are
-// dequantised to bf16 (q * s, rounded once) in registers inside the mainloop,
-// so no bf16 copy of an expert is ever written to global memory (ExactMoE
-// Section 3.1: the dequantised values define the operations; no FP16 expert is
-// materialised).
+// dequantised to bf16 (q * s exact in fp32, rounded once) in registers inside
+// the mainloop, so no bf16 copy of an expert is ever written to global memory
+// (ExactMoE Section 3.1: the dequantised values define the operations; no FP16
+// expert is materialised).
 //
-// Design (one persistent CTA per SM, 12 warps):
-//   warp 0  scheduler + TMA producer: takes work units from a global counter
-//           in descending cost class (BF16, then INT8, then INT4 experts),
-//           streams X tiles and BF16 weight tiles with TMA, INT8/INT4 packed
-//           tiles and their fp16 scales into a staging ring.
-//   warp 1  TMEM owner + MMA issuer: tcgen05.mma kind::f16, fp32 accumulators
-//           in TMEM, double-buffered so the epilogue overlaps the next unit.
-//   warps 4-7   epilogue: tcgen05.ld, SwiGLU (gate/up) or copy (down),
-//               bf16 stores.
-//   warps 8-11  dequant: staged INT8/INT4 codes x fp16 scale -> bf16 in the
-//               128-byte-swizzled K-major layout the tensor core reads.
-// A work unit is (expert, block of 256 weight rows, tile of <=128 rows).  For
-// gate/up the 256 weight rows are 128 gate rows and the matching 128 up rows,
-// so the epilogue sees g and u of the same feature.
+// Design (one persistent CTA per SM, 14 warps):
+//   warp 0       scheduler + TMA producer: takes work units from a global
+//                counter in descending cost class (BF16, then INT8, then INT4
+//                experts), streams X tiles and BF16 weight tiles with TMA, and
+//                INT8/INT4 codes plus their fp16 scales into a staging ring.
+//   warp 1       TMEM owner + MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16
+//                -> fp32) into double-buffered TMEM accumulators.
+//   warps 2,3,8-13  dequant: staged codes x scale -> bf16 in the 128-byte
+//                swizzled K-major layout the tensor core reads.
+//   warps 4-7    epilogue: tcgen05.ld, SwiGLU or copy, bf16 stores; overlaps
+//                the next unit's mainloop.
+// A work unit is (expert, block of weight rows, tile of <= 128 rows of that
+// expert).  Weight rows travel in 64-row TMA boxes; for gate/up a unit holds
+// matching gate and up boxes so one epilogue sees g and u of the same feature.
 //
-// Two MMA orientations:
-//   tile mode (kSwap = false, large groups): A = 128 token rows, B = 256 weight
-//     rows, D = 128 x 256 in TMEM; lane = token row.
-//   swap mode (kSwap = true, small groups, decode): A = 128 weight rows (two
-//     MMAs, one per half), B = the group's rows padded to 16, D = 2 x
-//     (128 x N); lane = weight row.  The tensor core then does no work on
-//     padding rows, so decode stays bound by weight bytes.
+// Two MMA orientations (the host picks one per launch from T = rows / k):
+//   tile mode (large groups, prefill): A = 128 token rows, B = 256 weight rows
+//     (128 gate + 128 up, or 256 down rows), D = 128 x 256 fp32; TMEM lane =
+//     token row.
+//   swap mode (small groups, decode): A = 128 weight rows (64 gate + 64 up, or
+//     128 down rows), B = the group's rows padded to 16, D = 128 x N; lane =
+//     weight row.  The tensor core does no work on padding rows and the small
+//     X tiles leave room for a deep weight pipeline, so decode streams weight
+//     bytes; the gate/up epilogue exchanges the up half through shared memory.
 #pragma once
 
 #include "common.cuh"
@@ -41,19 +43,19 @@
 namespace moe {
 namespace ffn {
 
-constexpr int kThreads = 384;
-constexpr int kNS = 3;                 // operand stages (64 K-elements each)
-constexpr int kNQ = 4;                 // staging slots for packed weights
-constexpr int kUR = 4;                 // work-unit ring depth
-constexpr int kWStage = 256 * 128;     // 256 weight rows x 128 B (64 bf16)
-constexpr int kXStage = 128 * 128;     // 128 rows x 128 B
-constexpr int kQSlot = 256 * 64;       // 256 rows x 64 B of packed codes
-constexpr int kQScale = 256 * 2;       // 256 fp16 scales
+constexpr int kThreads = 448;
+constexpr int kMaxNS = 8;          // operand stages (64 K-elements each)
+constexpr int kMaxNQ = 8;          // staging slots for packed weights
+constexpr int kUR = 4;             // work-unit ring depth
 constexpr int kMaxE = 512;
+constexpr int kBoxRows = 64;       // weight rows per TMA box
+constexpr int kDequantWarps = 8;   // warps 2, 3, 8 .. 13
+constexpr int kDequantThreads = 32 * kDequantWarps;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kSmemLimit = 232448; // dynamic shared memory per block on sm_100
 
 struct alignas(64) ExpertDesc {
-  CUtensorMap tm_w13;  // codes/values of [2I][H]; box 128 rows x (64 bf16 | 64 B)
+  CUtensorMap tm_w13;  // codes/values of [2I][H]; box 64 rows x (64 bf16 | 64 B)
   CUtensorMap tm_w2;   // codes/values of [H][I]
   const __half* s13;   // [H/128][2I]
   const __half* s2;    // [I/128][H]
@@ -63,80 +65,116 @@ struct alignas(64) ExpertDesc {
 static_assert(sizeof(ExpertDesc) == 320, "descriptor layout");
 
 struct Unit {
-  int e, prec, wrow0, nwh;  // expert, precision, first weight row, 128-row halves
+  int e, prec, wrow0, nbox;  // expert, precision, first weight row, 64-row boxes
   int row0, nrows, valid, pad;
 };
 
 struct Entry {
   int unit_begin;  // first unit index of this expert
-  int e;
+  int e_prec;      // expert id | precision << 16
   int row0;        // first permuted row of the expert
   int nrows;
 };
 
 struct Params {
   const ExpertDesc* descs;
+  const int* prec;         // [E] compact copy of descs[e].prec
   const int32_t* offsets;  // [E+1]
   __nv_bfloat16* out;      // h (gate/up) or y (down)
   int* counter;            // work counter, zero at launch
   int E, H, I;
   int K;          // reduction length: H (gate/up) or I (down)
   int out_ld;     // row stride of out: I (gate/up) or H (down)
-  int n_wblocks;  // I/128 (gate/up) or ceil(H/256) (down)
-  int xbox_rows;  // rows per X tensor-map box: 128 (tile mode) or 16 (swap mode)
+  int n_wblocks;  // weight blocks per expert
+  int xbox_rows;  // rows per X tensor-map box
+  int xrows;      // rows of an X stage = rows of a token tile (multiple of 16, <= 128)
+  int ns, nq;     // ring depths
 };
 
+// Shared-memory map (byte offsets from the 1024-aligned base).
+struct SmemMap {
+  uint32_t w, x, q, qs, xb, bar, units, misc, entries, total;
+  uint32_t wstage, xstage, qslot, qscale;
+};
+
+__host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows) {
+  SmemMap m;
+  const uint32_t wrows = swap ? 128 : 256;
+  m.wstage = wrows * 128;
+  m.xstage = (uint32_t)xrows * 128;
+  m.qslot = wrows * 64;
+  m.qscale = wrows * 2;
+  uint32_t off = 0;
+  m.w = off;
+  off += ns * m.wstage;
+  m.x = off;
+  off += ns * m.xstage;
+  m.q = off;
+  off += nq * m.qslot;
+  m.qs = off;
+  off += nq * m.qscale;
+  m.xb = off;
+  off += swap ? 64u * xrows * 4u : 0u;
+  off = (off + 15) & ~15u;
+  m.bar = off;
+  off += 64 * 8;
+  m.units = off;
+  off += kUR * sizeof(Unit);
+  m.misc = off;
+  off += 64;
+  m.entries = off;
+  off += kMaxE * sizeof(Entry);
+  m.total = off + 1024;  // slack to align the dynamic shared-memory base
+  return m;
+}
+
 struct Smem {
-  uint8_t* w_st;
-  uint8_t* x_st;
-  uint8_t* q_st;
-  uint8_t* q_sc;
-  uint64_t *full, *wfull, *empty, *qfull, *qempty, *accfull, *accempty, *ufull, *uempty, *mmadone;
+  uint8_t *w_st, *x_st, *q_st, *q_sc;
+  float* xbuf;
+  uint64_t *full, *wfull, *empty, *qfull, *qempty, *accfull, *accempty, *ufull, *uempty;
+  uint64_t *mmadone, *xfull, *xempty;
   Unit* units;
   uint32_t* tmem_slot;
   int* abort_flag;
   int* n_entries;
   int* n_units;
   Entry* entries;
+  uint32_t wstage, xstage, qslot, qscale;
 };
 
-__host__ __device__ constexpr size_t smem_bytes() {
-  return 1024 /* alignment slack */ + (size_t)kNS * kWStage + (size_t)kNS * kXStage +
-         (size_t)kNQ * kQSlot + (size_t)kNQ * kQScale + 64 * sizeof(uint64_t) /* barriers */ +
-         kUR * sizeof(Unit) + 64 /* misc words */ + (size_t)kMaxE * sizeof(Entry);
-}
-
-__device__ __forceinline__ Smem carve(uint8_t* raw) {
+__device__ __forceinline__ Smem carve(uint8_t* raw, const Params& p, bool swap) {
+  const SmemMap m = smem_map(swap, p.ns, p.nq, p.xrows);
+  uint8_t* b = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                          ~uintptr_t(1023));
   Smem s;
-  uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-  s.w_st = p;
-  p += kNS * kWStage;
-  s.x_st = p;
-  p += kNS * kXStage;
-  s.q_st = p;
-  p += kNQ * kQSlot;
-  s.q_sc = p;
-  p += kNQ * kQScale;
-  uint64_t* b = reinterpret_cast<uint64_t*>(p);
-  s.full = b;
-  s.wfull = s.full + kNS;
-  s.empty = s.wfull + kNS;
-  s.qfull = s.empty + kNS;
-  s.qempty = s.qfull + kNQ;
-  s.accfull = s.qempty + kNQ;
+  s.w_st = b + m.w;
+  s.x_st = b + m.x;
+  s.q_st = b + m.q;
+  s.q_sc = b + m.qs;
+  s.xbuf = reinterpret_cast<float*>(b + m.xb);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(b + m.bar);
+  s.full = bar;
+  s.wfull = s.full + kMaxNS;
+  s.empty = s.wfull + kMaxNS;
+  s.qfull = s.empty + kMaxNS;
+  s.qempty = s.qfull + kMaxNQ;
+  s.accfull = s.qempty + kMaxNQ;
   s.accempty = s.accfull + 2;
   s.ufull = s.accempty + 2;
   s.uempty = s.ufull + kUR;
   s.mmadone = s.uempty + kUR;
-  p += 64 * sizeof(uint64_t);
-  s.units = reinterpret_cast<Unit*>(p);
-  p += kUR * sizeof(Unit);
-  s.tmem_slot = reinterpret_cast<uint32_t*>(p);
-  s.abort_flag = reinterpret_cast<int*>(p + 4);
-  s.n_entries = reinterpret_cast<int*>(p + 8);
-  s.n_units = reinterpret_cast<int*>(p + 12);
-  p += 64;
-  s.entries = reinterpret_cast<Entry*>(p);
+  s.xfull = s.mmadone + 1;
+  s.xempty = s.xfull + 1;
+  s.units = reinterpret_cast<Unit*>(b + m.units);
+  s.tmem_slot = reinterpret_cast<uint32_t*>(b + m.misc);
+  s.abort_flag = reinterpret_cast<int*>(b + m.misc + 4);
+  s.n_entries = reinterpret_cast<int*>(b + m.misc + 8);
+  s.n_units = reinterpret_cast<int*>(b + m.misc + 12);
+  s.entries = reinterpret_cast<Entry*>(b + m.entries);
+  s.wstage = m.wstage;
+  s.xstage = m.xstage;
+  s.qslot = m.qslot;
+  s.qscale = m.qscale;
   return s;
 }
 
@@ -152,14 +190,28 @@ __device__ __forceinline__ void give_up(const Smem& s) {
   flag_status(MOE_STATUS_WAIT_TIMEOUT);
 }
 
-// Work units of one expert with n rows.
-__device__ __forceinline__ int units_of(int n, int n_wblocks) {
-  return n > 0 ? ((n + 127) / 128) * n_wblocks : 0;
+// Work units of one expert with n rows: token tiles of p.xrows rows (the X
+// stage's capacity) times weight blocks.
+__device__ __forceinline__ int units_of(int n, const Params& p) {
+  return n > 0 ? ((n + p.xrows - 1) / p.xrows) * p.n_wblocks : 0;
 }
 
-// Warp 0: list the experts with rows, cheapest-last (BF16 < INT8 < INT4 in
-// precision code = descending bytes per weight), with their first unit index.
+// All threads stage (offset, rows, precision) of every expert in shared memory
+// (one round of global loads), then warp 0 lists the experts with rows, most
+// bytes per weight first (BF16 < INT8 < INT4 in precision code), with their
+// first unit index.
 __device__ void build_entries(const Params& p, const Smem& s) {
+  int* t_off = reinterpret_cast<int*>(s.q_st);  // staging area is free until the mainloop
+  int* t_n = t_off + kMaxE;
+  int* t_prec = t_n + kMaxE;
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+    const int a = p.offsets[e], b = p.offsets[e + 1];
+    t_off[e] = a;
+    t_n[e] = b - a;
+    t_prec[e] = p.prec[e];
+  }
+  __syncthreads();
+  if ((threadIdx.x >> 5) != 0) return;
   const int lane = threadIdx.x & 31;
   const int per = (p.E + 31) / 32;
   const int e0 = lane * per;
@@ -170,11 +222,10 @@ __device__ void build_entries(const Params& p, const Smem& s) {
     for (int i = 0; i < per; ++i) {
       const int e = e0 + i;
       if (e >= p.E) break;
-      const int n = p.offsets[e + 1] - p.offsets[e];
-      const int prec = p.descs[e].prec;
+      const int n = t_n[e], prec = t_prec[e];
       if (cls == MOE_BF16 && n > 0 && (prec < MOE_BF16 || prec > MOE_INT4)) unset = true;
       if (prec == cls && n > 0) {
-        my_units += units_of(n, p.n_wblocks);
+        my_units += units_of(n, p);
         my_ents += 1;
       }
     }
@@ -192,10 +243,10 @@ __device__ void build_entries(const Params& p, const Smem& s) {
     for (int i = 0; i < per; ++i) {
       const int e = e0 + i;
       if (e >= p.E) break;
-      const int n = p.offsets[e + 1] - p.offsets[e];
-      if (p.descs[e].prec == cls && n > 0) {
-        s.entries[en] = Entry{u, e, p.offsets[e], n};
-        u += units_of(n, p.n_wblocks);
+      const int n = t_n[e];
+      if (t_prec[e] == cls && n > 0) {
+        s.entries[en] = Entry{u, e | (cls << 16), t_off[e], n};
+        u += units_of(n, p);
         en += 1;
       }
     }
@@ -209,7 +260,7 @@ __device__ void build_entries(const Params& p, const Smem& s) {
   }
 }
 
-template <bool kGateUp>
+template <bool kGateUp, bool kSwap>
 __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int u) {
   int lo = 0, hi = *s.n_entries - 1;  // last entry with unit_begin <= u
   while (lo < hi) {
@@ -223,46 +274,51 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
   const int local = u - en.unit_begin;
   const int tt = local / p.n_wblocks, wb = local % p.n_wblocks;
   Unit un;
-  un.e = en.e;
-  un.prec = p.descs[en.e].prec;
-  un.row0 = en.row0 + tt * 128;
-  un.nrows = min(128, en.nrows - tt * 128);
-  if (kGateUp) {
-    un.wrow0 = wb * 128;
-    un.nwh = 2;
+  un.e = en.e_prec & 0xFFFF;
+  un.prec = en.e_prec >> 16;
+  un.row0 = en.row0 + tt * p.xrows;
+  un.nrows = min(p.xrows, en.nrows - tt * p.xrows);
+  if (kGateUp) {  // gate rows [wrow0, wrow0 + rows/2), up rows I + the same
+    un.wrow0 = wb * (kSwap ? 64 : 128);
+    un.nbox = kSwap ? 2 : 4;
   } else {
-    un.wrow0 = wb * 256;
-    un.nwh = min(2, (p.H - un.wrow0) / 128);
+    un.wrow0 = wb * (kSwap ? 128 : 256);
+    un.nbox = min(kSwap ? 2 : 4, (p.H - un.wrow0) / kBoxRows);
   }
   un.valid = 1;
   un.pad = 0;
   return un;
 }
 
+// First weight row of 64-row box b of a unit.
 template <bool kGateUp>
-__device__ __forceinline__ int weight_row(const Params& p, const Unit& un, int h) {
-  return kGateUp ? (h == 0 ? un.wrow0 : p.I + un.wrow0) : un.wrow0 + 128 * h;
+__device__ __forceinline__ int box_row(const Params& p, const Unit& un, int b) {
+  if (!kGateUp) return un.wrow0 + kBoxRows * b;
+  const int half = un.nbox >> 1;  // boxes [0, half) gate, [half, nbox) up
+  return b < half ? un.wrow0 + kBoxRows * b : p.I + un.wrow0 + kBoxRows * (b - half);
 }
 
 // ---------------------------------------------------------------- producer --
 template <bool kGateUp, bool kSwap>
 __device__ void producer(const CUtensorMap* tm_x, const Params& p, const Smem& s) {
   volatile int* abort_flag = s.abort_flag;
+  const uint32_t ns = p.ns, nq = p.nq;
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
   uint32_t issued = 0, issued_par = 0, qissued = 0, qissued_par = 0;  // drain bookkeeping
   const int total = *s.n_units;
   const int nkb = p.K / 64;
   bool ok = true;
   prefetch_tmap(tm_x);
+  int next_u = atomicAdd(p.counter, 1);
   for (;;) {
     if (!mbar_wait(&s.uempty[us], uph ^ 1u, abort_flag)) {
       ok = false;
       break;
     }
-    const int u = atomicAdd(p.counter, 1);
+    const int u = next_u;
     Unit un;
     if (u < total) {
-      un = decode_unit<kGateUp>(p, s, u);
+      un = decode_unit<kGateUp, kSwap>(p, s, u);
     } else {
       un = Unit{0, 0, 0, 0, 0, 0, 0, 0};
     }
@@ -277,9 +333,11 @@ __device__ void producer(const CUtensorMap* tm_x, const Params& p, const Smem& s
     const int srows = kGateUp ? 2 * p.I : p.H;  // rows of the scale matrix
     tmap_acquire(tw);
     prefetch_tmap(tw);
-    const int nxb = kSwap ? (un.nrows + p.xbox_rows - 1) / p.xbox_rows : 1;
+    const int nxb = (un.nrows + p.xbox_rows - 1) / p.xbox_rows;
     const uint32_t xbytes = (uint32_t)(nxb * p.xbox_rows * 128);
-    for (int kb = 0; kb < nkb && ok; ++kb) {
+    const int prefetch_kb = max(0, nkb - (int)ns);  // reserve the next unit near the end
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (kb == prefetch_kb) next_u = atomicAdd(p.counter, 1);
       if (!mbar_wait(&s.empty[st], sph ^ 1u, abort_flag)) {
         ok = false;
         break;
@@ -289,39 +347,41 @@ __device__ void producer(const CUtensorMap* tm_x, const Params& p, const Smem& s
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&s.qfull[q], (uint32_t)un.nwh * (128 * 64 + 256));
+        mbar_arrive_expect_tx(&s.qfull[q], (uint32_t)un.nbox * (kBoxRows * 64 + kBoxRows * 2));
         const int kc = (un.prec == MOE_INT8) ? kb * 64 : (kb >> 1) * 64;  // byte column
         const int g = kb >> 1;                                             // K-group
-        for (int h = 0; h < un.nwh; ++h) {
-          const int wr = weight_row<kGateUp>(p, un, h);
-          tma_load_2d(s.q_st + q * kQSlot + h * 8192, tw, kc, wr, &s.qfull[q]);
-          bulk_load(s.q_sc + q * kQScale + h * 256, sc + (size_t)g * srows + wr, 256, &s.qfull[q]);
+        for (int b = 0; b < un.nbox; ++b) {
+          const int wr = box_row<kGateUp>(p, un, b);
+          tma_load_2d(s.q_st + q * s.qslot + b * (kBoxRows * 64), tw, kc, wr, &s.qfull[q]);
+          bulk_load(s.q_sc + q * s.qscale + b * (kBoxRows * 2), sc + (size_t)g * srows + wr,
+                    kBoxRows * 2, &s.qfull[q]);
         }
         qissued |= 1u << q;
         qissued_par = (qissued_par & ~(1u << q)) | (qph << q);
-        advance(q, qph, kNQ);
+        advance(q, qph, nq);
       }
-      const uint32_t bytes = xbytes + (un.prec == MOE_BF16 ? (uint32_t)un.nwh * 16384u : 0u);
+      const uint32_t bytes =
+          xbytes + (un.prec == MOE_BF16 ? (uint32_t)un.nbox * (kBoxRows * 128) : 0u);
       mbar_arrive_expect_tx(&s.full[st], bytes);
       for (int b = 0; b < nxb; ++b)
-        tma_load_2d(s.x_st + st * kXStage + b * p.xbox_rows * 128, tm_x, kb * 64,
+        tma_load_2d(s.x_st + st * s.xstage + b * p.xbox_rows * 128, tm_x, kb * 64,
                     un.row0 + b * p.xbox_rows, &s.full[st]);
       if (un.prec == MOE_BF16)
-        for (int h = 0; h < un.nwh; ++h)
-          tma_load_2d(s.w_st + st * kWStage + h * 16384, tw, kb * 64, weight_row<kGateUp>(p, un, h),
-                      &s.full[st]);
+        for (int b = 0; b < un.nbox; ++b)
+          tma_load_2d(s.w_st + st * s.wstage + b * (kBoxRows * 128), tw, kb * 64,
+                      box_row<kGateUp>(p, un, b), &s.full[st]);
       issued |= 1u << st;
       issued_par = (issued_par & ~(1u << st)) | (sph << st);
-      advance(st, sph, kNS);
+      advance(st, sph, ns);
     }
     if (!ok) break;
   }
   if (!ok) {
     give_up(s);
     // Let copies already in flight land before the CTA's shared memory goes away.
-    for (uint32_t i = 0; i < (uint32_t)kNS; ++i)
+    for (uint32_t i = 0; i < ns; ++i)
       if (issued & (1u << i)) mbar_wait(&s.full[i], (issued_par >> i) & 1u);
-    for (uint32_t i = 0; i < (uint32_t)kNQ; ++i)
+    for (uint32_t i = 0; i < nq; ++i)
       if (qissued & (1u << i)) mbar_wait(&s.qfull[i], (qissued_par >> i) & 1u);
   }
 }
@@ -330,6 +390,7 @@ __device__ void producer(const CUtensorMap* tm_x, const Params& p, const Smem& s
 template <bool kGateUp, bool kSwap>
 __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
   volatile int* abort_flag = s.abort_flag;
+  const uint32_t ns = p.ns;
   uint32_t st = 0, sph = 0, us = 0, uph = 0, abuf = 0;
   uint32_t aph[2] = {0, 0};
   uint32_t wph = 0;  // wfull phase bit per stage: it only advances on INT8/INT4 units
@@ -349,9 +410,9 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
       break;
     }
     tc_fence_after();
-    const uint32_t d_base = tmem + abuf * 256;
-    const int nmma = kSwap ? max(16, (un.nrows + 15) & ~15) : un.nwh * 128;
-    const uint32_t idesc = idesc_bf16_f32(128, nmma);
+    const uint32_t d_tmem = tmem + abuf * 256;
+    const int n = kSwap ? max(16, (un.nrows + 15) & ~15) : un.nbox * kBoxRows;
+    const uint32_t idesc = idesc_bf16_f32(128, n);
     const bool quant = un.prec != MOE_BF16;
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mbar_wait(&s.full[st], sph, abort_flag) ||
@@ -361,22 +422,20 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
       }
       if (quant) wph ^= 1u << st;
       tc_fence_after();
-      const uint32_t xa = smem_u32(s.x_st + st * kXStage);
-      const uint32_t wa = smem_u32(s.w_st + st * kWStage);
+      const uint32_t xa = smem_u32(s.x_st + st * s.xstage);
+      const uint32_t wa = smem_u32(s.w_st + st * s.wstage);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint32_t acc = (kb | kk) != 0;
-        if (kSwap) {
-          for (int h = 0; h < un.nwh; ++h)
-            mma_bf16_ss(d_base + h * 128, smem_desc_sw128(wa + h * 16384 + kk * 32),
-                        smem_desc_sw128(xa + kk * 32), idesc, acc);
-        } else {
-          mma_bf16_ss(d_base, smem_desc_sw128(xa + kk * 32), smem_desc_sw128(wa + kk * 32), idesc,
+        if (kSwap)
+          mma_bf16_ss(d_tmem, smem_desc_sw128(wa + kk * 32), smem_desc_sw128(xa + kk * 32), idesc,
                       acc);
-        }
+        else
+          mma_bf16_ss(d_tmem, smem_desc_sw128(xa + kk * 32), smem_desc_sw128(wa + kk * 32), idesc,
+                      acc);
       }
       mma_commit(&s.empty[st]);
-      advance(st, sph, kNS);
+      advance(st, sph, ns);
     }
     if (!ok) break;
     mma_commit(&s.accfull[abuf]);
@@ -390,18 +449,57 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
 }
 
 // ----------------------------------------------------------------- dequant --
-// 128 threads convert one 64-element K-slice of up to 256 weight rows: thread
-// (row r = tid/8 + 16 i, 16-byte chunk c = tid % 8) -> 8 bf16 at the swizzled
-// position of chunk c in row r.  Each warp signals its own part (barrier
-// counts are 4), so the four warps never wait on one another.
+// Code -> bf16 dequantisation, exact up to the final rounding.  A code byte u
+// (INT4: the nibble, u = q + 8; INT8: the byte xor 0x80, u = q + 128) becomes
+// the fp32 m = 2^15 + u by placing it in mantissa bits 8..15 of 2^15 (one
+// prmt).  Then fma(m, s, -(2^15 + off) * s) = (u - off) * s = q * s, where the
+// constant is exact in fp32 ((2^15 + 8) * s needs 24 bits, (2^15 + 128) * s
+// 20 bits, s being fp16) and the fused product-sum is rounded once, so the
+// fp32 result is q * s exactly; cvt.rn.bf16x2 then rounds it to bf16.
+__device__ __forceinline__ uint32_t place_byte(uint32_t src, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0x47000000, %2;" : "=r"(d) : "r"(src), "r"(sel));
+  return d;
+}
+
+// Two codes (byte b0 of src0, byte b1 of src1) -> packed bf16x2 of q * s.
+__device__ __forceinline__ uint32_t deq2(uint32_t src0, uint32_t sel0, uint32_t src1,
+                                         uint32_t sel1, uint64_t s2, uint64_t c2) {
+  uint64_t m, w;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(m) : "r"(place_byte(src0, sel0)), "r"(place_byte(src1, sel1)));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(w) : "l"(m), "l"(s2), "l"(c2));
+  uint32_t lo, hi, d;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(w));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "r"(hi), "r"(lo));
+  return d;
+}
+
+// prmt selector that puts byte b of the first operand into bits 8..15 over
+// 0x47000000 (bytes 0 and 2 zero, byte 3 = 0x47).
+__device__ __forceinline__ constexpr uint32_t sel_byte(uint32_t b) { return 0x7604u | (b << 4); }
+
+__device__ __forceinline__ uint64_t f32x2(float v) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+  return r;
+}
+
+// One staging slot holds an INT4 group (128 K-elements = two k-blocks) or an
+// INT8 k-block (64 K-elements) for the unit's weight rows, 64 bytes per row.
+// Work item = 16 bytes of codes of one row: INT4 -> 32 elements (4 output
+// chunks of 8), INT8 -> 16 elements (2 chunks).  A thread loads all its items
+// first, then converts and stores them in the 128-byte-swizzled K-major layout
+// (chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)).  Each warp signals
+// its own part (barrier counts are kDequantWarps), so the warps never wait on
+// one another.
 template <bool kGateUp>
-__device__ void dequant(const Params& p, const Smem& s) {
+__device__ void dequant(const Params& p, const Smem& s, int dtid) {
   volatile int* abort_flag = s.abort_flag;
-  const int tid = threadIdx.x - 256;  // 0..127
   const int lane = threadIdx.x & 31;
-  const int c = tid & 7, rsub = tid >> 3;
+  const uint32_t ns = p.ns, nq = p.nq;
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
   const int nkb = p.K / 64;
+  constexpr int kMaxItems = 4;  // 256 rows x 4 items / kDequantThreads
   bool ok = true;
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
@@ -414,50 +512,81 @@ __device__ void dequant(const Params& p, const Smem& s) {
     advance(us, uph, kUR);
     if (!un.valid) break;
     if (un.prec == MOE_BF16) {
-      for (int kb = 0; kb < nkb; ++kb) advance(st, sph, kNS);
+      for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
       continue;
     }
-    const int rows = un.nwh * 128;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const bool first = un.prec == MOE_INT8 || (kb & 1) == 0;
-      const bool last = un.prec == MOE_INT8 || (kb & 1) == 1;
-      if ((first && !mbar_wait(&s.qfull[q], qph, abort_flag)) ||
-          !mbar_wait(&s.empty[st], sph ^ 1u, abort_flag)) {
+    const bool int4 = un.prec == MOE_INT4;
+    const int items = un.nbox * kBoxRows * 4;
+    const float off = int4 ? 32776.0f : 32896.0f;  // 2^15 + 8, 2^15 + 128
+    const uint32_t flip = int4 ? 0u : 0x80808080u;
+    for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
+      const uint32_t st0 = st, sph0 = sph;
+      advance(st, sph, ns);
+      const uint32_t st1 = st, sph1 = sph;
+      if (int4) advance(st, sph, ns);
+      if (!mbar_wait(&s.qfull[q], qph, abort_flag) ||
+          !mbar_wait(&s.empty[st0], sph0 ^ 1u, abort_flag) ||
+          (int4 && !mbar_wait(&s.empty[st1], sph1 ^ 1u, abort_flag))) {
         ok = false;
         break;
       }
-      const uint8_t* qs = s.q_st + q * kQSlot;
-      const __half* scs = reinterpret_cast<const __half*>(s.q_sc + q * kQScale);
-      const uint32_t wdst = smem_u32(s.w_st + st * kWStage);
-      for (int r = rsub; r < rows; r += 16) {
-        const int h = r >> 7, rr = r & 127;
-        const float sc = __half2float(scs[h * 128 + rr]);
-        const uint8_t* src = qs + h * 8192 + rr * 64;
-        float f[8];
-        if (un.prec == MOE_INT4) {
-          const uint32_t v = *reinterpret_cast<const uint32_t*>(src + (kb & 1) * 32 + c * 4);
+      const uint8_t* qs = s.q_st + q * s.qslot;
+      const __half* scs = reinterpret_cast<const __half*>(s.q_sc + q * s.qscale);
+      const uint32_t w0 = smem_u32(s.w_st + st0 * s.wstage);
+      const uint32_t w1 = smem_u32(s.w_st + st1 * s.wstage);
+      uint4 code[kMaxItems];
+      float sc[kMaxItems];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)  // (2^23 + u) - (2^23 + 8) = u - 8 = q, exact
-            f[j] = (__uint_as_float(0x4B000000u | ((v >> (4 * j)) & 0xFu)) - 8388616.0f) * sc;
+      for (int i = 0; i < kMaxItems; ++i) {
+        const int it = dtid + i * kDequantThreads;
+        if (it < items) {
+          code[i] = *reinterpret_cast<const uint4*>(qs + it * 16);  // row it/4, quarter it%4
+          sc[i] = __half2float(scs[it >> 2]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kMaxItems; ++i) {
+        const int it = dtid + i * kDequantThreads;
+        if (it >= items) break;
+        const int r = it >> 2, qq = it & 3;
+        const uint64_t s2 = f32x2(sc[i]), c2 = f32x2(-off * sc[i]);
+        const uint32_t wv[4] = {code[i].x, code[i].y, code[i].z, code[i].w};
+        const uint32_t rbase = (uint32_t)r * 128;
+        if (int4) {
+          // elements 32 qq .. 32 qq + 31 of the group: k-block half qq / 2,
+          // chunks 4 (qq % 2) .. + 3; word j holds chunk j's 8 nibbles
+          const uint32_t dst = ((qq >> 1) ? w1 : w0) + rbase;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t lo = wv[j] & 0x0F0F0F0Fu, hi = (wv[j] >> 4) & 0x0F0F0F0Fu;
+            const int c = (qq & 1) * 4 + j;
+            st_shared_v4(dst + ((c ^ (r & 7)) << 4), deq2(lo, sel_byte(0), hi, sel_byte(0), s2, c2),
+                         deq2(lo, sel_byte(1), hi, sel_byte(1), s2, c2),
+                         deq2(lo, sel_byte(2), hi, sel_byte(2), s2, c2),
+                         deq2(lo, sel_byte(3), hi, sel_byte(3), s2, c2));
+          }
         } else {
-          const uint2 v = *reinterpret_cast<const uint2*>(src + c * 8);
+          // elements 16 qq .. 16 qq + 15 of the k-block: chunks 2 qq, 2 qq + 1
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {  // (2^23 + q + 128) - (2^23 + 128) = q, exact
-            const uint32_t b = ((j < 4 ? v.x : v.y) >> (8 * (j & 3))) & 0xFFu;
-            f[j] = (__uint_as_float(0x4B000000u | (b ^ 0x80u)) - 8388736.0f) * sc;
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t a = wv[2 * j] ^ flip, b = wv[2 * j + 1] ^ flip;
+            const int c = qq * 2 + j;
+            st_shared_v4(w0 + rbase + ((c ^ (r & 7)) << 4),
+                         deq2(a, sel_byte(0), a, sel_byte(1), s2, c2),
+                         deq2(a, sel_byte(2), a, sel_byte(3), s2, c2),
+                         deq2(b, sel_byte(0), b, sel_byte(1), s2, c2),
+                         deq2(b, sel_byte(2), b, sel_byte(3), s2, c2));
           }
         }
-        st_shared_v4(wdst + r * 128 + ((c ^ (r & 7)) << 4), pack_bf16x2(f[0], f[1]),
-                     pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {  // one arrival per dequant warp (barrier counts are 4)
-        mbar_arrive(&s.wfull[st]);
-        if (last) mbar_arrive(&s.qempty[q]);
+      if (lane == 0) {  // one arrival per dequant warp and stage
+        mbar_arrive(&s.wfull[st0]);
+        if (int4) mbar_arrive(&s.wfull[st1]);
+        mbar_arrive(&s.qempty[q]);
       }
-      if (last) advance(q, qph, kNQ);
-      advance(st, sph, kNS);
+      advance(q, qph, nq);
     }
     if (!ok) break;
   }
@@ -472,7 +601,7 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
   volatile int* abort_flag = s.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-  uint32_t us = 0, uph = 0, ebuf = 0;
+  uint32_t us = 0, uph = 0, ebuf = 0, xph = 0;
   uint32_t eph[2] = {0, 0};
   bool ok = true;
   for (;;) {
@@ -492,37 +621,60 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
     tc_fence_after();
     const uint32_t tb = tmem + ((uint32_t)(quarter * 32) << 16) + ebuf * 256;
     if (kSwap) {
-      const int wr = quarter * 32 + lane;  // weight row inside a 128-row half
+      const int wr = quarter * 32 + lane;  // weight row of the unit (TMEM lane)
       const int n_pad = max(16, (un.nrows + 15) & ~15);
-      for (int n0 = 0; n0 < n_pad; n0 += 16) {
-        if (kGateUp) {
-          uint32_t g[16], u[16];
-          tmem_ld16(tb + n0, g);
-          tmem_ld16(tb + 128 + n0, u);
-          tmem_ld_wait();
+      if (kGateUp) {
+        // lanes 0-63: gate rows, lanes 64-127: the matching up rows
+        if (quarter >= 2) {
+          if (!mbar_wait(s.xempty, xph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          for (int n0 = 0; n0 < n_pad; n0 += 16) {
+            uint32_t u[16];
+            tmem_ld16(tb + n0, u);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (n0 + j < un.nrows)
-              p.out[(size_t)(un.row0 + n0 + j) * p.out_ld + un.wrow0 + wr] =
-                  __float2bfloat16_rn(silu_mul(__uint_as_float(g[j]), __uint_as_float(u[j])));
+            for (int j = 0; j < 16; ++j) s.xbuf[(n0 + j) * 64 + (wr - 64)] = __uint_as_float(u[j]);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s.xfull);
         } else {
-          for (int h = 0; h < un.nwh; ++h) {
-            uint32_t v[16];
-            tmem_ld16(tb + h * 128 + n0, v);
+          if (!mbar_wait(s.xfull, xph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          for (int n0 = 0; n0 < n_pad; n0 += 16) {
+            uint32_t gv[16];
+            tmem_ld16(tb + n0, gv);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               if (n0 + j < un.nrows)
-                p.out[(size_t)(un.row0 + n0 + j) * p.out_ld + un.wrow0 + h * 128 + wr] =
-                    __float2bfloat16_rn(__uint_as_float(v[j]));
+                p.out[(size_t)(un.row0 + n0 + j) * p.out_ld + un.wrow0 + wr] = __float2bfloat16_rn(
+                    silu_mul(__uint_as_float(gv[j]), s.xbuf[(n0 + j) * 64 + wr]));
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s.xempty);
+        }
+        xph ^= 1u;
+      } else {
+        for (int n0 = 0; n0 < n_pad; n0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tb + n0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (n0 + j < un.nrows && wr < un.nbox * kBoxRows)
+              p.out[(size_t)(un.row0 + n0 + j) * p.out_ld + un.wrow0 + wr] =
+                  __float2bfloat16_rn(__uint_as_float(v[j]));
         }
       }
     } else {
       const int m = quarter * 32 + lane;  // token row inside the tile
       const bool valid = m < un.nrows;
       uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)(un.row0 + m) * p.out_ld + un.wrow0);
-      const int ncols = kGateUp ? 128 : un.nwh * 128;
+      const int ncols = kGateUp ? 128 : un.nbox * kBoxRows;
       for (int c0 = 0; c0 < ncols; c0 += 16) {
         uint32_t a[16], b[16];
         tmem_ld16(tb + c0, a);
@@ -555,18 +707,18 @@ template <bool kGateUp, bool kSwap>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_ffn_kernel(const __grid_constant__ CUtensorMap tm_x, const Params p) {
   extern __shared__ uint8_t ffn_smem_raw[];
-  const Smem s = carve(ffn_smem_raw);
+  const Smem s = carve(ffn_smem_raw, p, kSwap);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNS; ++i) {
-      mbar_init(&s.full[i], 1);   // producer's arrive.expect_tx
-      mbar_init(&s.wfull[i], 4);  // one arrival per dequant warp
-      mbar_init(&s.empty[i], 1);  // tcgen05.commit
+    for (int i = 0; i < kMaxNS; ++i) {
+      mbar_init(&s.full[i], 1);                // producer's arrive.expect_tx
+      mbar_init(&s.wfull[i], kDequantWarps);   // one arrival per dequant warp
+      mbar_init(&s.empty[i], 1);               // tcgen05.commit
     }
-    for (int i = 0; i < kNQ; ++i) {
+    for (int i = 0; i < kMaxNQ; ++i) {
       mbar_init(&s.qfull[i], 1);
-      mbar_init(&s.qempty[i], 4);
+      mbar_init(&s.qempty[i], kDequantWarps);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.accfull[i], 1);
@@ -574,9 +726,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kUR; ++i) {
       mbar_init(&s.ufull[i], 1);
-      mbar_init(&s.uempty[i], 9);  // MMA thread + 4 epilogue warps + 4 dequant warps
+      mbar_init(&s.uempty[i], 1 + 4 + kDequantWarps);  // MMA thread + epilogue + dequant warps
     }
     mbar_init(s.mmadone, 1);
+    mbar_init(s.xfull, 2);   // the two epilogue warps holding the up half
+    mbar_init(s.xempty, 2);  // the two epilogue warps holding the gate half
     *s.abort_flag = 0;
     fence_mbar_init();
   }
@@ -584,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(s.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0) build_entries(p, s);
+  build_entries(p, s);  // contains a __syncthreads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -596,8 +750,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mma_issuer<kGateUp, kSwap>(p, s, tmem);
   } else if (warp >= 4 && warp < 8) {
     epilogue<kGateUp, kSwap>(p, s, tmem);
-  } else if (warp >= 8) {
-    dequant<kGateUp>(p, s);
+  } else {
+    const int dtid = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // warps 2, 3, 8 .. 13
+    dequant<kGateUp>(p, s, dtid);
   }
 
   tc_fence_before();
@@ -607,11 +762,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Stream-ordered install of one expert descriptor (a by-value kernel argument,
-// so the host buffer needs no lifetime beyond the launch).
-__global__ void write_desc_kernel(ExpertDesc* dst, const __grid_constant__ ExpertDesc d) {
+// so the host buffer needs no lifetime beyond the launch) and of its precision
+// in the compact precision array.
+__global__ void write_desc_kernel(ExpertDesc* dst, int* prec_dst,
+                                  const __grid_constant__ ExpertDesc d) {
   const int i = threadIdx.x;
   if (i < (int)(sizeof(ExpertDesc) / 16))
     reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(&d)[i];
+  if (i == 0) *prec_dst = d.prec;
   tmap_release();
 }
 

@@ -88,14 +88,15 @@ int encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int e
 }
 
 // Tensor map of one expert weight matrix [rows][K] in its storage format:
-// BF16 -> box 128 rows x 64 bf16 (128-byte swizzle, the MMA operand layout);
-// INT8/INT4 -> box 128 rows x 64 bytes of codes (staged, then dequantised).
+// BF16 -> box 64 rows x 64 bf16 (128-byte swizzle, the MMA operand layout);
+// INT8/INT4 -> box 64 rows x 64 bytes of codes (staged, then dequantised).
 int encode_weight(CUtensorMap* m, const void* base, int prec, int rows, int K) {
+  const uint32_t box_rows = moe::ffn::kBoxRows;
   if (prec == MOE_BF16)
-    return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 128, 64,
+    return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, box_rows, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B);
   const int cols = (prec == MOE_INT4) ? K / 2 : K;
-  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, 128, 64,
+  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, box_rows, 64,
                    CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
@@ -111,6 +112,7 @@ struct moe_layer {
   int H, I, E, k;
   int device;
   moe::ffn::ExpertDesc* d_descs;  // [E], device
+  int* d_prec;                    // [E], device: compact copy of the precisions
   std::vector<int> prec;          // host shadow, -1 = unset
 };
 
@@ -130,16 +132,18 @@ int moe_layer_create(int H, int I, int E, int k, moe_layer_t* out) {
   int dev = 0;
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   moe::ffn::ExpertDesc* d = nullptr;
-  MOE_CUDA_TRY(cudaMalloc(&d, sizeof(moe::ffn::ExpertDesc) * E));
-  // All bytes 0xFF: prec = -1 (unset) for every expert.
-  cudaError_t e1 = cudaMemset(d, 0xFF, sizeof(moe::ffn::ExpertDesc) * E);
+  const size_t table = sizeof(moe::ffn::ExpertDesc) * E;
+  MOE_CUDA_TRY(cudaMalloc(&d, table + sizeof(int) * E));
+  int* dp = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(d) + table);
+  // All bytes 0xFF: prec = -1 (unset) for every expert, in both arrays.
+  cudaError_t e1 = cudaMemset(d, 0xFF, table + sizeof(int) * E);
   cudaError_t e2 = cudaDeviceSynchronize();
   if (e1 != cudaSuccess || e2 != cudaSuccess) {
     cudaFree(d);
     return fail(MOE_ERR_CUDA, "descriptor table init failed: %s",
                 cudaGetErrorString(e1 != cudaSuccess ? e1 : e2));
   }
-  moe_layer* L = new moe_layer{H, I, E, k, dev, d, std::vector<int>(E, -1)};
+  moe_layer* L = new moe_layer{H, I, E, k, dev, d, dp, std::vector<int>(E, -1)};
   *out = L;
   return ok();
 }
@@ -179,7 +183,8 @@ int moe_set_expert_precision(moe_layer_t L, int expert, moe_precision_t precisio
   d.s13 = prec == MOE_BF16 ? nullptr : static_cast<const __half*>(w->s13);
   d.s2 = prec == MOE_BF16 ? nullptr : static_cast<const __half*>(w->s2);
   d.prec = prec;
-  moe::ffn::write_desc_kernel<<<1, 32, 0, as_stream(stream)>>>(L->d_descs + expert, d);
+  moe::ffn::write_desc_kernel<<<1, 32, 0, as_stream(stream)>>>(L->d_descs + expert,
+                                                               L->d_prec + expert, d);
   MOE_CUDA_TRY(cudaGetLastError());
   L->prec[expert] = prec;
   return ok();
@@ -294,10 +299,17 @@ int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expe
   int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + need - 256);
   MOE_CUDA_TRY(cudaMemsetAsync(counters, 0, 2 * sizeof(int), s));
 
-  // Every expert holds at most T = rows / k rows; up to 128 rows fit one swap-mode tile.
+  // Every expert holds at most T = rows / k rows.  Small groups (decode) use the
+  // weights-as-M orientation with a deep pipeline sized for the largest group.
   const int T = (rows + L->k - 1) / L->k;
   const bool swap = T <= 128;
   const int xbox = swap ? 16 : 128;
+  const int xrows = swap ? std::max(16, (std::min(T, 128) + 15) / 16 * 16) : 128;
+  const int nq = swap ? 6 : 4;
+  int ns = kMaxNS;
+  while (ns > 2 && (int)smem_map(swap, ns, nq, xrows).total > kSmemLimit) --ns;
+  const int smem = (int)smem_map(swap, ns, nq, xrows).total;
+  MOE_CHECK(smem <= kSmemLimit, MOE_ERR_UNSUPPORTED, "shared memory plan does not fit");
 
   CUtensorMap tm_x, tm_h;
   int rc = encode_2d(&tm_x, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->H, xbox, 64,
@@ -307,21 +319,22 @@ int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expe
                  CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != MOE_OK) return rc;
 
-  Params pg{L->d_descs, expert_offsets, h, counters, L->E, L->H, L->I, L->H, L->I, L->I / 128, xbox};
-  Params pd{L->d_descs, expert_offsets, static_cast<__nv_bfloat16*>(y_perm), counters + 1, L->E,
-            L->H, L->I, L->I, L->H, (L->H + 255) / 256, xbox};
+  Params pg{L->d_descs, L->d_prec, expert_offsets, h, counters, L->E, L->H, L->I, L->H, L->I,
+            swap ? L->I / 64 : L->I / 128, xbox, xrows, ns, nq};
+  Params pd{L->d_descs, L->d_prec, expert_offsets, static_cast<__nv_bfloat16*>(y_perm),
+            counters + 1, L->E, L->H, L->I, L->I, L->H, swap ? L->H / 128 : (L->H + 255) / 256,
+            xbox, xrows, ns, nq};
 
   static bool attr_set = false;
-  const int smem = (int)smem_bytes();
   if (!attr_set) {
     MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<true, true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<false, true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<true, false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<false, false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     attr_set = true;
   }
   if (swap) {
