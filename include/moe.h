@@ -150,7 +150,8 @@ int moe_ffn_workspace_bytes(moe_layer_t layer, int rows, size_t* bytes);
  *   rows           T*k, the row capacity of x_perm / y_perm
  *   y_perm         device bf16 [rows][H]; rows >= offsets[E] are not written
  *   workspace      device, >= moe_ffn_workspace_bytes(rows) bytes, 256-byte
- *                  aligned; holds h and the tile scheduler's counters.
+ *                  aligned; holds h and the tile scheduler's counters (zeroed
+ *                  by the call itself).
  * Fails with MOE_ERR_NOT_MATERIALIZED if any expert was never set.  Calls that
  * share a workspace must not overlap on the device. */
 int moe_grouped_ffn_mixed(moe_layer_t layer, const void* x_perm,

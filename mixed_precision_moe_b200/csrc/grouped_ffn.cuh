@@ -1,31 +1,38 @@
 // grouped_ffn.cuh -- mixed-precision grouped SwiGLU expert FFN for sm_100a.
 //
-// One launch computes, for every expert e and every permuted row r of e,
-// either the fused gate/up projection with the SwiGLU epilogue
-//     h_r = silu(x_r W_g,e^T) * (x_r W_u,e^T)
-// or the down projection  y_r = h_r W_d,e^T  (ExactMoE, Section 3.4: "one
-// fused gate/up projection and one down projection" per group of experts).
-// Experts in one launch may be BF16, INT8 or INT4 (MxMoE abstract: GEMMs of
-// different precisions in one grouped kernel); INT8/INT4 weights are
-// dequantised to bf16 (q * s exact in fp32, rounded once) in registers inside
-// the mainloop, so no bf16 copy of an expert is ever written to global memory
-// (ExactMoE Section 3.1: the dequantised values define the operations; no FP16
-// expert is materialised).
+// One persistent launch computes the whole expert FFN: for every expert e and
+// every permuted row r of e, the fused gate/up projection with the SwiGLU
+// epilogue  h_r = silu(x_r W_g,e^T) * (x_r W_u,e^T)  and then the down
+// projection  y_r = h_r W_d,e^T  (ExactMoE, Section 3.4: one fused gate/up
+// projection and one down projection per group of experts).  Experts in one
+// launch may be BF16, INT8 or INT4 (MxMoE abstract: GEMMs of different
+// precisions in one grouped kernel); INT8/INT4 weights are dequantised to bf16
+// (q * s exact in fp32, rounded once) in registers inside the mainloop, so no
+// bf16 copy of an expert is ever written to global memory (ExactMoE Section
+// 3.1: the dequantised values define the operations; no FP16 expert is
+// materialised).
 //
-// Design (one persistent CTA per SM, 14 warps):
+// Design (one persistent CTA per SM, 15 warps):
 //   warp 0       scheduler + TMA producer: takes work units from a global
-//                counter in descending cost class (BF16, then INT8, then INT4
-//                experts), streams X tiles and BF16 weight tiles with TMA, and
-//                INT8/INT4 codes plus their fp16 scales into a staging ring.
+//                counter -- every gate/up unit, then every down unit, each in
+//                descending time per unit (INT4/INT8 experts before BF16) --
+//                and streams X tiles and BF16 weight tiles with TMA.  A down
+//                unit first waits (bounded) until all gate/up epilogues of its
+//                expert have published their h rows.
+//   warp 14      code producer: streams INT8/INT4 codes and their fp16 scales
+//                into a staging ring, running ahead of the operand stages.
 //   warp 1       TMEM owner + MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16
 //                -> fp32) into double-buffered TMEM accumulators.
-//   warps 2,3,8-13  dequant: staged codes x scale -> bf16 in the 128-byte
-//                swizzled K-major layout the tensor core reads.
-//   warps 4-7    epilogue: tcgen05.ld, SwiGLU or copy, bf16 stores; overlaps
-//                the next unit's mainloop.
-// A work unit is (expert, block of weight rows, tile of <= 128 rows of that
-// expert).  Weight rows travel in 64-row TMA boxes; for gate/up a unit holds
-// matching gate and up boxes so one epilogue sees g and u of the same feature.
+//   warps 2,3,8-13  dequant: staged codes x scale -> bf16, into shared memory
+//                (tile mode) or straight into TMEM as the MMA's A operand
+//                (swap mode).
+//   warps 4-7    epilogue: tcgen05.ld, SwiGLU or copy, bf16 stores; gate/up
+//                epilogues publish their rows with a release counter.
+// A work unit is (projection, expert, block of weight rows, tile of rows of
+// that expert).  Weight rows travel in 64-row TMA boxes; for gate/up a unit
+// holds matching gate and up boxes so one epilogue sees g and u of the same
+// feature.  Running both projections in one launch needs one prologue instead
+// of two, and down units fill the tail of the gate/up phase.
 //
 // Two MMA orientations (the host picks one per launch from T = rows / k):
 //   tile mode (large groups, prefill): A = 128 token rows, B = 256 weight rows
@@ -43,7 +50,7 @@
 namespace moe {
 namespace ffn {
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kMaxNS = 8;          // operand stages (64 K-elements each)
 constexpr int kMaxNQ = 8;          // staging slots for packed weights
 constexpr int kUR = 4;             // work-unit ring depth
@@ -66,11 +73,14 @@ static_assert(sizeof(ExpertDesc) == 320, "descriptor layout");
 
 struct Unit {
   int e, prec, wrow0, nbox;  // expert, precision, first weight row, 64-row boxes
-  int row0, nrows, valid, pad;
+  int row0, nrows;           // rows of the token tile
+  int flags;                 // kUnitValid | kUnitGateUp
+  int need;                  // down unit: gate/up epilogue arrivals to wait for
 };
+constexpr int kUnitValid = 1, kUnitGateUp = 2;
 
 struct Entry {
-  int unit_begin;  // first unit index of this expert
+  int unit_begin;  // first gate/up unit index of this expert
   int e_prec;      // expert id | precision << 16
   int row0;        // first permuted row of the expert
   int nrows;
@@ -80,15 +90,15 @@ struct Params {
   const ExpertDesc* descs;
   const int* prec;         // [E] compact copy of descs[e].prec
   const int32_t* offsets;  // [E+1]
-  __nv_bfloat16* out;      // h (gate/up) or y (down)
+  __nv_bfloat16* h;        // [rows][I]: gate/up output, down input
+  __nv_bfloat16* y;        // [rows][H]: down output
   int* counter;            // work counter, zero at launch
+  int* done;               // [E] finished gate/up epilogue warps per expert, zero at launch
   int E, H, I;
-  int K;          // reduction length: H (gate/up) or I (down)
-  int out_ld;     // row stride of out: I (gate/up) or H (down)
-  int n_wblocks;  // weight blocks per expert
-  int xbox_rows;  // rows per X tensor-map box
-  int xrows;      // rows of an X stage = rows of a token tile (multiple of 16, <= 128)
-  int ns, nq;     // ring depths
+  int nwb_gu, nwb_dn;      // weight blocks per expert of each projection
+  int xbox_rows;           // rows per X tensor-map box
+  int xrows;               // rows of an X stage = rows of a token tile (multiple of 16, <= 128)
+  int ns, nq;              // ring depths
 };
 
 // Shared-memory map (byte offsets from the 1024-aligned base).
@@ -123,7 +133,7 @@ __host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows
   m.misc = off;
   off += 64;
   m.entries = off;
-  off += kMaxE * sizeof(Entry);
+  off += kMaxE * sizeof(Entry) + kMaxE * sizeof(int);  // entries, then first down unit
   m.total = off + 1024;  // slack to align the dynamic shared-memory base
   return m;
 }
@@ -138,7 +148,9 @@ struct Smem {
   int* abort_flag;
   int* n_entries;
   int* n_units;
+  int* n_units_gu;
   Entry* entries;
+  int* ub_dn;  // [entry] first down unit of the entry's expert
   uint32_t wstage, xstage, qslot, qscale;
 };
 
@@ -170,7 +182,9 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const Params& p, bool swap) 
   s.abort_flag = reinterpret_cast<int*>(b + m.misc + 4);
   s.n_entries = reinterpret_cast<int*>(b + m.misc + 8);
   s.n_units = reinterpret_cast<int*>(b + m.misc + 12);
+  s.n_units_gu = reinterpret_cast<int*>(b + m.misc + 16);
   s.entries = reinterpret_cast<Entry*>(b + m.entries);
+  s.ub_dn = reinterpret_cast<int*>(b + m.entries + kMaxE * sizeof(Entry));
   s.wstage = m.wstage;
   s.xstage = m.xstage;
   s.qslot = m.qslot;
@@ -190,16 +204,19 @@ __device__ __forceinline__ void give_up(const Smem& s) {
   flag_status(MOE_STATUS_WAIT_TIMEOUT);
 }
 
-// Work units of one expert with n rows: token tiles of p.xrows rows (the X
-// stage's capacity) times weight blocks.
-__device__ __forceinline__ int units_of(int n, const Params& p) {
-  return n > 0 ? ((n + p.xrows - 1) / p.xrows) * p.n_wblocks : 0;
+// Token tiles of an expert with n rows (tiles of p.xrows rows, the X stage's
+// capacity); each tile is paired with every weight block of a projection.
+__device__ __forceinline__ int tiles_of(int n, const Params& p) {
+  return n > 0 ? (n + p.xrows - 1) / p.xrows : 0;
 }
 
 // All threads stage (offset, rows, precision) of every expert in shared memory
-// (one round of global loads), then warp 0 lists the experts with rows, most
-// bytes per weight first (BF16 < INT8 < INT4 in precision code), with their
-// first unit index.
+// (one round of global loads), then warp 0 lists the experts with rows, with
+// their first unit index, in descending time per unit: INT4 and INT8 units
+// (dequant- and latency-bound) before BF16 units, so the dynamic scheduler
+// approximates longest-processing-time-first and the tail is made of the
+// short units.  Unit indices: every gate/up unit in that order, then every
+// down unit in the same expert order.
 __device__ void build_entries(const Params& p, const Smem& s) {
   int* t_off = reinterpret_cast<int*>(s.q_st);  // staging area is free until the mainloop
   int* t_n = t_off + kMaxE;
@@ -215,100 +232,147 @@ __device__ void build_entries(const Params& p, const Smem& s) {
   const int lane = threadIdx.x & 31;
   const int per = (p.E + 31) / 32;
   const int e0 = lane * per;
-  int unit_run = 0, ent_run = 0;
+  int tile_run = 0, ent_run = 0;
   bool unset = false;
-  for (int cls = MOE_BF16; cls <= MOE_INT4; ++cls) {
-    int my_units = 0, my_ents = 0;
+  constexpr int kClassOrder[3] = {MOE_INT4, MOE_INT8, MOE_BF16};
+  for (int ci = 0; ci < 3; ++ci) {
+    const int cls = kClassOrder[ci];
+    int my_tiles = 0, my_ents = 0;
     for (int i = 0; i < per; ++i) {
       const int e = e0 + i;
       if (e >= p.E) break;
       const int n = t_n[e], prec = t_prec[e];
-      if (cls == MOE_BF16 && n > 0 && (prec < MOE_BF16 || prec > MOE_INT4)) unset = true;
+      if (ci == 0 && n > 0 && (prec < MOE_BF16 || prec > MOE_INT4)) unset = true;
       if (prec == cls && n > 0) {
-        my_units += units_of(n, p);
+        my_tiles += tiles_of(n, p);
         my_ents += 1;
       }
     }
-    int u_incl = my_units, e_incl = my_ents;
+    int t_incl = my_tiles, e_incl = my_ents;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, u_incl, d);
+      const int a = __shfl_up_sync(0xffffffffu, t_incl, d);
       const int b = __shfl_up_sync(0xffffffffu, e_incl, d);
       if (lane >= d) {
-        u_incl += a;
+        t_incl += a;
         e_incl += b;
       }
     }
-    int u = unit_run + u_incl - my_units, en = ent_run + e_incl - my_ents;
+    int t = tile_run + t_incl - my_tiles, en = ent_run + e_incl - my_ents;
     for (int i = 0; i < per; ++i) {
       const int e = e0 + i;
       if (e >= p.E) break;
       const int n = t_n[e];
       if (t_prec[e] == cls && n > 0) {
-        s.entries[en] = Entry{u, e | (cls << 16), t_off[e], n};
-        u += units_of(n, p);
+        // tiles before this expert, times the weight blocks of each projection
+        s.entries[en] = Entry{t * p.nwb_gu, e | (cls << 16), t_off[e], n};
+        s.ub_dn[en] = t * p.nwb_dn;  // offset by the gate/up total below
+        t += tiles_of(n, p);
         en += 1;
       }
     }
-    unit_run += __shfl_sync(0xffffffffu, u_incl, 31);
+    tile_run += __shfl_sync(0xffffffffu, t_incl, 31);
     ent_run += __shfl_sync(0xffffffffu, e_incl, 31);
   }
+  const int total_gu = tile_run * p.nwb_gu;
+  __syncwarp();
+  for (int i = lane; i < ent_run; i += 32) s.ub_dn[i] += total_gu;
   if (__any_sync(0xffffffffu, unset) && lane == 0) flag_status(MOE_STATUS_UNSET_EXPERT);
   if (lane == 0) {
-    *s.n_units = unit_run;
+    *s.n_units_gu = total_gu;
+    *s.n_units = total_gu + tile_run * p.nwb_dn;
     *s.n_entries = ent_run;
   }
 }
 
-template <bool kGateUp, bool kSwap>
+template <bool kSwap>
 __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int u) {
-  int lo = 0, hi = *s.n_entries - 1;  // last entry with unit_begin <= u
+  const bool gu = u < *s.n_units_gu;
+  int lo = 0, hi = *s.n_entries - 1;  // last entry whose first unit is <= u
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (s.entries[mid].unit_begin <= u)
+    if ((gu ? s.entries[mid].unit_begin : s.ub_dn[mid]) <= u)
       lo = mid;
     else
       hi = mid - 1;
   }
   const Entry en = s.entries[lo];
-  const int local = u - en.unit_begin;
-  const int tt = local / p.n_wblocks, wb = local % p.n_wblocks;
+  const int nwb = gu ? p.nwb_gu : p.nwb_dn;
+  const int local = u - (gu ? en.unit_begin : s.ub_dn[lo]);
+  const int tt = local / nwb, wb = local % nwb;
   Unit un;
   un.e = en.e_prec & 0xFFFF;
   un.prec = en.e_prec >> 16;
   un.row0 = en.row0 + tt * p.xrows;
   un.nrows = min(p.xrows, en.nrows - tt * p.xrows);
-  if (kGateUp) {  // gate rows [wrow0, wrow0 + rows/2), up rows I + the same
+  if (gu) {  // gate rows [wrow0, wrow0 + rows/2), up rows I + the same
     un.wrow0 = wb * (kSwap ? 64 : 128);
     un.nbox = kSwap ? 2 : 4;
   } else {
     un.wrow0 = wb * (kSwap ? 128 : 256);
     un.nbox = min(kSwap ? 2 : 4, (p.H - un.wrow0) / kBoxRows);
   }
-  un.valid = 1;
-  un.pad = 0;
+  un.flags = kUnitValid | (gu ? kUnitGateUp : 0);
+  un.need = 4 * tiles_of(en.nrows, p) * p.nwb_gu;  // 4 epilogue warps per gate/up unit
   return un;
 }
 
+__device__ __forceinline__ bool unit_gu(const Unit& un) { return (un.flags & kUnitGateUp) != 0; }
+
 // First weight row of 64-row box b of a unit.
-template <bool kGateUp>
 __device__ __forceinline__ int box_row(const Params& p, const Unit& un, int b) {
-  if (!kGateUp) return un.wrow0 + kBoxRows * b;
+  if (!unit_gu(un)) return un.wrow0 + kBoxRows * b;
   const int half = un.nbox >> 1;  // boxes [0, half) gate, [half, nbox) up
   return b < half ? un.wrow0 + kBoxRows * b : p.I + un.wrow0 + kBoxRows * (b - half);
 }
 
+// Reduction length of the unit's projection in 64-element k-blocks.
+__device__ __forceinline__ int unit_nkb(const Params& p, const Unit& un) {
+  return (unit_gu(un) ? p.H : p.I) / 64;
+}
+
+__device__ __forceinline__ int ld_acquire(const int* ptr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(int* ptr, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Down unit: wait until every gate/up epilogue warp of the expert has
+// published its h rows (bounded), then order those generic-proxy writes before
+// this thread's TMA (async-proxy) reads.
+__device__ __forceinline__ bool wait_gate_up(const Params& p, const Unit& un,
+                                             volatile int* abort_flag) {
+  const int* cnt = p.done + un.e;
+  const long long t0 = clock64();
+  while (ld_acquire(cnt) < un.need) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+    __nanosleep(128);
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
 // ---------------------------------------------------------------- producer --
-template <bool kGateUp, bool kSwap>
-__device__ void producer(const CUtensorMap* tm_x, const Params& p, const Smem& s) {
+template <bool kSwap>
+__device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const Params& p,
+                         const Smem& s) {
   volatile int* abort_flag = s.abort_flag;
-  const uint32_t ns = p.ns, nq = p.nq;
-  uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
-  uint32_t issued = 0, issued_par = 0, qissued = 0, qissued_par = 0;  // drain bookkeeping
+  const uint32_t ns = p.ns;
+  uint32_t st = 0, sph = 0, us = 0, uph = 0;
+  uint32_t issued = 0, issued_par = 0;  // drain bookkeeping
   const int total = *s.n_units;
-  const int nkb = p.K / 64;
   bool ok = true;
   prefetch_tmap(tm_x);
+  prefetch_tmap(tm_h);
   int next_u = atomicAdd(p.counter, 1);
   for (;;) {
     if (!mbar_wait(&s.uempty[us], uph ^ 1u, abort_flag)) {
@@ -318,21 +382,28 @@ __device__ void producer(const CUtensorMap* tm_x, const Params& p, const Smem& s
     const int u = next_u;
     Unit un;
     if (u < total) {
-      un = decode_unit<kGateUp, kSwap>(p, s, u);
+      un = decode_unit<kSwap>(p, s, u);
     } else {
       un = Unit{0, 0, 0, 0, 0, 0, 0, 0};
     }
     s.units[us] = un;
     mbar_arrive(&s.ufull[us]);
     advance(us, uph, kUR);
-    if (!un.valid) break;
+    if (!(un.flags & kUnitValid)) break;
 
+    const bool gu = unit_gu(un);
     const ExpertDesc* d = p.descs + un.e;
-    const CUtensorMap* tw = kGateUp ? &d->tm_w13 : &d->tm_w2;
-    const __half* sc = kGateUp ? d->s13 : d->s2;
-    const int srows = kGateUp ? 2 * p.I : p.H;  // rows of the scale matrix
-    tmap_acquire(tw);
-    prefetch_tmap(tw);
+    const CUtensorMap* tw = gu ? &d->tm_w13 : &d->tm_w2;
+    const CUtensorMap* tx = gu ? tm_x : tm_h;
+    if (un.prec == MOE_BF16) {
+      tmap_acquire(tw);
+      prefetch_tmap(tw);
+    }
+    if (!gu && !wait_gate_up(p, un, abort_flag)) {
+      ok = false;
+      break;
+    }
+    const int nkb = unit_nkb(p, un);
     const int nxb = (un.nrows + p.xbox_rows - 1) / p.xbox_rows;
     const uint32_t xbytes = (uint32_t)(nxb * p.xbox_rows * 128);
     const int prefetch_kb = max(0, nkb - (int)ns);  // reserve the next unit near the end
@@ -342,34 +413,16 @@ __device__ void producer(const CUtensorMap* tm_x, const Params& p, const Smem& s
         ok = false;
         break;
       }
-      if (un.prec != MOE_BF16 && (un.prec == MOE_INT8 || (kb & 1) == 0)) {
-        if (!mbar_wait(&s.qempty[q], qph ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&s.qfull[q], (uint32_t)un.nbox * (kBoxRows * 64 + kBoxRows * 2));
-        const int kc = (un.prec == MOE_INT8) ? kb * 64 : (kb >> 1) * 64;  // byte column
-        const int g = kb >> 1;                                             // K-group
-        for (int b = 0; b < un.nbox; ++b) {
-          const int wr = box_row<kGateUp>(p, un, b);
-          tma_load_2d(s.q_st + q * s.qslot + b * (kBoxRows * 64), tw, kc, wr, &s.qfull[q]);
-          bulk_load(s.q_sc + q * s.qscale + b * (kBoxRows * 2), sc + (size_t)g * srows + wr,
-                    kBoxRows * 2, &s.qfull[q]);
-        }
-        qissued |= 1u << q;
-        qissued_par = (qissued_par & ~(1u << q)) | (qph << q);
-        advance(q, qph, nq);
-      }
       const uint32_t bytes =
           xbytes + (un.prec == MOE_BF16 ? (uint32_t)un.nbox * (kBoxRows * 128) : 0u);
       mbar_arrive_expect_tx(&s.full[st], bytes);
       for (int b = 0; b < nxb; ++b)
-        tma_load_2d(s.x_st + st * s.xstage + b * p.xbox_rows * 128, tm_x, kb * 64,
+        tma_load_2d(s.x_st + st * s.xstage + b * p.xbox_rows * 128, tx, kb * 64,
                     un.row0 + b * p.xbox_rows, &s.full[st]);
       if (un.prec == MOE_BF16)
         for (int b = 0; b < un.nbox; ++b)
           tma_load_2d(s.w_st + st * s.wstage + b * (kBoxRows * 128), tw, kb * 64,
-                      box_row<kGateUp>(p, un, b), &s.full[st]);
+                      box_row(p, un, b), &s.full[st]);
       issued |= 1u << st;
       issued_par = (issued_par & ~(1u << st)) | (sph << st);
       advance(st, sph, ns);
@@ -381,20 +434,18 @@ __device__ void producer(const CUtensorMap* tm_x, const Params& p, const Smem& s
     // Let copies already in flight land before the CTA's shared memory goes away.
     for (uint32_t i = 0; i < ns; ++i)
       if (issued & (1u << i)) mbar_wait(&s.full[i], (issued_par >> i) & 1u);
-    for (uint32_t i = 0; i < nq; ++i)
-      if (qissued & (1u << i)) mbar_wait(&s.qfull[i], (qissued_par >> i) & 1u);
   }
 }
 
-// -------------------------------------------------------------- MMA issuer --
-template <bool kGateUp, bool kSwap>
-__device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
+// ------------------------------------------------------------ code producer --
+// Streams the INT8/INT4 codes and fp16 scales of each quantised unit into the
+// staging ring, as far ahead as the ring allows, independently of the operand
+// stages (which wait on the tensor core); BF16 units are skipped.
+__device__ void code_producer(const Params& p, const Smem& s) {
   volatile int* abort_flag = s.abort_flag;
-  const uint32_t ns = p.ns;
-  uint32_t st = 0, sph = 0, us = 0, uph = 0, abuf = 0;
-  uint32_t aph[2] = {0, 0};
-  uint32_t wph = 0;  // wfull phase bit per stage: it only advances on INT8/INT4 units
-  const int nkb = p.K / 64;
+  const uint32_t nq = p.nq;
+  uint32_t q = 0, qph = 0, us = 0, uph = 0;
+  uint32_t qissued = 0, qissued_par = 0;  // drain bookkeeping
   bool ok = true;
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
@@ -404,16 +455,79 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
     const Unit un = s.units[us];
     mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
-    if (!un.valid) break;
+    if (!(un.flags & kUnitValid)) break;
+    if (un.prec == MOE_BF16) continue;
+    const bool gu = unit_gu(un);
+    const ExpertDesc* d = p.descs + un.e;
+    const CUtensorMap* tw = gu ? &d->tm_w13 : &d->tm_w2;
+    const __half* sc = gu ? d->s13 : d->s2;
+    const int srows = gu ? 2 * p.I : p.H;  // rows of the scale matrix
+    tmap_acquire(tw);
+    prefetch_tmap(tw);
+    const int nkb = unit_nkb(p, un);
+    const bool int4 = un.prec == MOE_INT4;
+    for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
+      if (!mbar_wait(&s.qempty[q], qph ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&s.qfull[q], (uint32_t)un.nbox * (kBoxRows * 64 + kBoxRows * 2));
+      const int kc = int4 ? (kb >> 1) * 64 : kb * 64;  // byte column of the codes
+      const int g = kb >> 1;                            // K-group of the scales
+      for (int b = 0; b < un.nbox; ++b) {
+        const int wr = box_row(p, un, b);
+        tma_load_2d(s.q_st + q * s.qslot + b * (kBoxRows * 64), tw, kc, wr, &s.qfull[q]);
+        bulk_load(s.q_sc + q * s.qscale + b * (kBoxRows * 2), sc + (size_t)g * srows + wr,
+                  kBoxRows * 2, &s.qfull[q]);
+      }
+      qissued |= 1u << q;
+      qissued_par = (qissued_par & ~(1u << q)) | (qph << q);
+      advance(q, qph, nq);
+    }
+    if (!ok) break;
+  }
+  if (!ok) {
+    give_up(s);
+    for (uint32_t i = 0; i < nq; ++i)
+      if (qissued & (1u << i)) mbar_wait(&s.qfull[i], (qissued_par >> i) & 1u);
+  }
+}
+
+// -------------------------------------------------------------- MMA issuer --
+// TMEM columns: tile mode uses two 256-column accumulators; swap mode uses two
+// 128-column accumulators (N <= 128) and, from column kATmemCol, one 32-column
+// A stage per operand stage (64 K-elements x 128 rows of dequantised weights).
+constexpr uint32_t kATmemCol = 256;
+
+template <bool kSwap>
+__device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
+  constexpr uint32_t kAccCols = kSwap ? 128 : 256;
+  volatile int* abort_flag = s.abort_flag;
+  const uint32_t ns = p.ns;
+  uint32_t st = 0, sph = 0, us = 0, uph = 0, abuf = 0;
+  uint32_t aph[2] = {0, 0};
+  uint32_t wph = 0;  // wfull phase bit per stage: it only advances on INT8/INT4 units
+  bool ok = true;
+  for (;;) {
+    if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
+      ok = false;
+      break;
+    }
+    const Unit un = s.units[us];
+    mbar_arrive(&s.uempty[us]);
+    advance(us, uph, kUR);
+    if (!(un.flags & kUnitValid)) break;
+    const int nkb = unit_nkb(p, un);
     if (!mbar_wait(&s.accempty[abuf], aph[abuf] ^ 1u, abort_flag)) {
       ok = false;
       break;
     }
     tc_fence_after();
-    const uint32_t d_tmem = tmem + abuf * 256;
+    const uint32_t d_tmem = tmem + abuf * kAccCols;
     const int n = kSwap ? max(16, (un.nrows + 15) & ~15) : un.nbox * kBoxRows;
     const uint32_t idesc = idesc_bf16_f32(128, n);
     const bool quant = un.prec != MOE_BF16;
+    const bool a_in_tmem = kSwap && quant;  // dequantised weights live in TMEM
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mbar_wait(&s.full[st], sph, abort_flag) ||
           (quant && !mbar_wait(&s.wfull[st], (wph >> st) & 1u, abort_flag))) {
@@ -427,7 +541,10 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint32_t acc = (kb | kk) != 0;
-        if (kSwap)
+        if (a_in_tmem)
+          mma_bf16_ts(d_tmem, tmem + kATmemCol + st * 32 + kk * 8, smem_desc_sw128(xa + kk * 32),
+                      idesc, acc);
+        else if (kSwap)
           mma_bf16_ss(d_tmem, smem_desc_sw128(wa + kk * 32), smem_desc_sw128(xa + kk * 32), idesc,
                       acc);
         else
@@ -492,13 +609,95 @@ __device__ __forceinline__ uint64_t f32x2(float v) {
 // (chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)).  Each warp signals
 // its own part (barrier counts are kDequantWarps), so the warps never wait on
 // one another.
-template <bool kGateUp>
+// Swap mode: dequantised weights go to TMEM instead of shared memory.  Warp w
+// owns TMEM lane quarter w % 4 (= weight rows 32 (w % 4) .. + 31 of the unit,
+// one row per thread) and one half of each staging slot (warps 10..13 the
+// second half): INT4 slot = two k-blocks (half h -> k-block 2g + h, 32 code
+// bytes -> 64 elements -> 32 columns), INT8 slot = one k-block (half h ->
+// elements 32 h .. + 31 -> 16 columns).
+__device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
+  volatile int* abort_flag = s.abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int half = warp >= 10 ? 1 : 0;
+  const int r = quarter * 32 + lane;  // weight row of the unit = TMEM lane
+  const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + kATmemCol;
+  const uint32_t ns = p.ns, nq = p.nq;
+  uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
+  bool ok = true;
+  for (;;) {
+    if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
+      ok = false;
+      break;
+    }
+    const Unit un = s.units[us];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.uempty[us]);
+    advance(us, uph, kUR);
+    if (!(un.flags & kUnitValid)) break;
+    const int nkb = unit_nkb(p, un);
+    if (un.prec == MOE_BF16) {
+      for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
+      continue;
+    }
+    const bool int4 = un.prec == MOE_INT4;
+    const float off = int4 ? 32776.0f : 32896.0f;  // 2^15 + 8, 2^15 + 128
+    for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
+      const uint32_t st0 = st, sph0 = sph;
+      advance(st, sph, ns);
+      const uint32_t st1 = st, sph1 = sph;
+      if (int4) advance(st, sph, ns);
+      if (!mbar_wait(&s.qfull[q], qph, abort_flag) ||
+          !mbar_wait(&s.empty[st0], sph0 ^ 1u, abort_flag) ||
+          (int4 && !mbar_wait(&s.empty[st1], sph1 ^ 1u, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint4* src = reinterpret_cast<const uint4*>(s.q_st + q * s.qslot + r * 64 + half * 32);
+      const uint4 c0 = src[0], c1 = src[1];
+      const float sc = __half2float(reinterpret_cast<const __half*>(s.q_sc + q * s.qscale)[r]);
+      const uint64_t s2 = f32x2(sc), k2 = f32x2(-off * sc);
+      const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      if (int4) {
+        uint32_t v[32];  // word j = elements 8 j .. 8 j + 7 -> columns 4 j .. 4 j + 3
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t lo = w[j] & 0x0F0F0F0Fu, hi = (w[j] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) v[4 * j + b] = deq2(lo, sel_byte(b), hi, sel_byte(b), s2, k2);
+        }
+        tmem_st32(lane_addr + (half ? st1 : st0) * 32, v);
+      } else {
+        uint32_t v[16];  // word j = elements 4 j .. 4 j + 3 -> columns 2 j, 2 j + 1
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t a = w[j] ^ 0x80808080u;
+          v[2 * j] = deq2(a, sel_byte(0), a, sel_byte(1), s2, k2);
+          v[2 * j + 1] = deq2(a, sel_byte(2), a, sel_byte(3), s2, k2);
+        }
+        tmem_st16(lane_addr + st0 * 32 + half * 16, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {  // one arrival per dequant warp and stage
+        mbar_arrive(&s.wfull[st0]);
+        if (int4) mbar_arrive(&s.wfull[st1]);
+        mbar_arrive(&s.qempty[q]);
+      }
+      advance(q, qph, nq);
+    }
+    if (!ok) break;
+  }
+  if (!ok) give_up(s);
+}
+
 __device__ void dequant(const Params& p, const Smem& s, int dtid) {
   volatile int* abort_flag = s.abort_flag;
   const int lane = threadIdx.x & 31;
   const uint32_t ns = p.ns, nq = p.nq;
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
-  const int nkb = p.K / 64;
   constexpr int kMaxItems = 4;  // 256 rows x 4 items / kDequantThreads
   bool ok = true;
   for (;;) {
@@ -510,7 +709,8 @@ __device__ void dequant(const Params& p, const Smem& s, int dtid) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
-    if (!un.valid) break;
+    if (!(un.flags & kUnitValid)) break;
+    const int nkb = unit_nkb(p, un);
     if (un.prec == MOE_BF16) {
       for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
       continue;
@@ -596,8 +796,19 @@ __device__ void dequant(const Params& p, const Smem& s, int dtid) {
 // ---------------------------------------------------------------- epilogue --
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-template <bool kGateUp, bool kSwap>
+// Gate/up epilogue: once this warp's h stores are done, publish them to the
+// down units of the expert (release counter; the proxy fence orders the
+// generic-proxy stores before any TMA read that the counter enables).
+__device__ __forceinline__ void publish_rows(const Params& p, const Unit& un, int lane) {
+  fence_proxy_async_global();
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) red_release_add(p.done + un.e, 1);
+}
+
+template <bool kSwap>
 __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
+  constexpr uint32_t kAccCols = kSwap ? 128 : 256;
   volatile int* abort_flag = s.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
@@ -613,17 +824,18 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
-    if (!un.valid) break;
+    if (!(un.flags & kUnitValid)) break;
+    const bool gu = unit_gu(un);
     if (!mbar_wait(&s.accfull[ebuf], eph[ebuf], abort_flag)) {
       ok = false;
       break;
     }
     tc_fence_after();
-    const uint32_t tb = tmem + ((uint32_t)(quarter * 32) << 16) + ebuf * 256;
+    const uint32_t tb = tmem + ((uint32_t)(quarter * 32) << 16) + ebuf * kAccCols;
     if (kSwap) {
       const int wr = quarter * 32 + lane;  // weight row of the unit (TMEM lane)
       const int n_pad = max(16, (un.nrows + 15) & ~15);
-      if (kGateUp) {
+      if (gu) {
         // lanes 0-63: gate rows, lanes 64-127: the matching up rows
         if (quarter >= 2) {
           if (!mbar_wait(s.xempty, xph ^ 1u, abort_flag)) {
@@ -651,7 +863,7 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               if (n0 + j < un.nrows)
-                p.out[(size_t)(un.row0 + n0 + j) * p.out_ld + un.wrow0 + wr] = __float2bfloat16_rn(
+                p.h[(size_t)(un.row0 + n0 + j) * p.I + un.wrow0 + wr] = __float2bfloat16_rn(
                     silu_mul(__uint_as_float(gv[j]), s.xbuf[(n0 + j) * 64 + wr]));
           }
           __syncwarp();
@@ -666,25 +878,26 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (n0 + j < un.nrows && wr < un.nbox * kBoxRows)
-              p.out[(size_t)(un.row0 + n0 + j) * p.out_ld + un.wrow0 + wr] =
+              p.y[(size_t)(un.row0 + n0 + j) * p.H + un.wrow0 + wr] =
                   __float2bfloat16_rn(__uint_as_float(v[j]));
         }
       }
     } else {
       const int m = quarter * 32 + lane;  // token row inside the tile
       const bool valid = m < un.nrows;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)(un.row0 + m) * p.out_ld + un.wrow0);
-      const int ncols = kGateUp ? 128 : un.nbox * kBoxRows;
+      __nv_bfloat16* out = gu ? p.h + (size_t)(un.row0 + m) * p.I + un.wrow0
+                              : p.y + (size_t)(un.row0 + m) * p.H + un.wrow0;
+      uint4* dst = reinterpret_cast<uint4*>(out);
+      const int ncols = gu ? 128 : un.nbox * kBoxRows;
       for (int c0 = 0; c0 < ncols; c0 += 16) {
         uint32_t a[16], b[16];
         tmem_ld16(tb + c0, a);
-        if (kGateUp) tmem_ld16(tb + 128 + c0, b);
+        if (gu) tmem_ld16(tb + 128 + c0, b);
         tmem_ld_wait();
         float f[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          f[j] = kGateUp ? silu_mul(__uint_as_float(a[j]), __uint_as_float(b[j]))
-                         : __uint_as_float(a[j]);
+          f[j] = gu ? silu_mul(__uint_as_float(a[j]), __uint_as_float(b[j])) : __uint_as_float(a[j]);
         if (valid) {
           dst[c0 / 8] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                                    pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
@@ -696,6 +909,7 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.accempty[ebuf]);
+    if (gu) publish_rows(p, un, lane);
     eph[ebuf] ^= 1u;
     ebuf ^= 1u;
   }
@@ -703,41 +917,43 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
 }
 
 // ------------------------------------------------------------------ kernel --
-template <bool kGateUp, bool kSwap>
+template <bool kSwap>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_ffn_kernel(const __grid_constant__ CUtensorMap tm_x, const Params p) {
+    grouped_ffn_kernel(const __grid_constant__ CUtensorMap tm_x,
+                       const __grid_constant__ CUtensorMap tm_h, const Params p) {
   extern __shared__ uint8_t ffn_smem_raw[];
   const Smem s = carve(ffn_smem_raw, p, kSwap);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kMaxNS; ++i) {
+  {  // barrier initialisation, one barrier per thread of warps 2 and 3
+    const int i = threadIdx.x - 64;
+    if (i >= 0 && i < kMaxNS) {
       mbar_init(&s.full[i], 1);                // producer's arrive.expect_tx
       mbar_init(&s.wfull[i], kDequantWarps);   // one arrival per dequant warp
       mbar_init(&s.empty[i], 1);               // tcgen05.commit
+    } else if (i >= kMaxNS && i < kMaxNS + kMaxNQ) {
+      mbar_init(&s.qfull[i - kMaxNS], 1);
+      mbar_init(&s.qempty[i - kMaxNS], kDequantWarps);
+    } else if (i >= 16 && i < 18) {
+      mbar_init(&s.accfull[i - 16], 1);
+      mbar_init(&s.accempty[i - 16], 4);
+    } else if (i >= 18 && i < 18 + kUR) {
+      mbar_init(&s.ufull[i - 18], 1);
+      mbar_init(&s.uempty[i - 18], 2 + 4 + kDequantWarps);  // MMA, code producer, epilogue, dequant
+    } else if (i == 30) {
+      mbar_init(s.mmadone, 1);
+      mbar_init(s.xfull, 2);   // the two epilogue warps holding the up half
+      mbar_init(s.xempty, 2);  // the two epilogue warps holding the gate half
+      *s.abort_flag = 0;
     }
-    for (int i = 0; i < kMaxNQ; ++i) {
-      mbar_init(&s.qfull[i], 1);
-      mbar_init(&s.qempty[i], kDequantWarps);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.accfull[i], 1);
-      mbar_init(&s.accempty[i], 4);
-    }
-    for (int i = 0; i < kUR; ++i) {
-      mbar_init(&s.ufull[i], 1);
-      mbar_init(&s.uempty[i], 1 + 4 + kDequantWarps);  // MMA thread + epilogue + dequant warps
-    }
-    mbar_init(s.mmadone, 1);
-    mbar_init(s.xfull, 2);   // the two epilogue warps holding the up half
-    mbar_init(s.xempty, 2);  // the two epilogue warps holding the gate half
-    *s.abort_flag = 0;
-    fence_mbar_init();
+    if (i >= 0 && i < 32) fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(s.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  pdl_launch_dependents();
+  pdl_wait();           // inputs of the previous kernels are complete from here on
   build_entries(p, s);  // contains a __syncthreads
   tc_fence_before();
   __syncthreads();
@@ -745,14 +961,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *s.tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) producer<kGateUp, kSwap>(&tm_x, p, s);
+    if (lane == 0) producer<kSwap>(&tm_x, &tm_h, p, s);
   } else if (warp == 1) {
-    if (lane == 0) mma_issuer<kGateUp, kSwap>(p, s, tmem);
+    if (lane == 0) mma_issuer<kSwap>(p, s, tmem);
   } else if (warp >= 4 && warp < 8) {
-    epilogue<kGateUp, kSwap>(p, s, tmem);
+    epilogue<kSwap>(p, s, tmem);
+  } else if (warp == 14) {
+    if (lane == 0) code_producer(p, s);
   } else {
-    const int dtid = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // warps 2, 3, 8 .. 13
-    dequant<kGateUp>(p, s, dtid);
+    if (kSwap) {
+      dequant_tmem(p, s, tmem);
+    } else {
+      const int dtid = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // warps 2, 3, 8 .. 13
+      dequant(p, s, dtid);
+    }
   }
 
   tc_fence_before();

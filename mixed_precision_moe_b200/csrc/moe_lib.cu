@@ -8,6 +8,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "common.cuh"
@@ -99,6 +100,30 @@ int encode_weight(CUtensorMap* m, const void* base, int prec, int rows, int K) {
   return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, box_rows, 64,
                    CU_TENSOR_MAP_SWIZZLE_NONE);
 }
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while its predecessor in the stream drains; the kernels themselves execute
+// griddepcontrol.wait before reading anything a predecessor wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Scheduler counters at the end of the FFN workspace: the work counter, then
+// (from int 16) one gate/up completion counter per expert.
+constexpr size_t kFfnCounterBytes = 4096;
+size_t ffn_counter_bytes(int E) { return (16 + (size_t)E) * sizeof(int); }
 
 int num_sms(int device) {
   int n = 0;
@@ -208,17 +233,12 @@ int moe_route_topk(const float* logits, int T, int E, int k, int renormalize, in
   const int keys = (E + 31) / 32;
   const dim3 block(256), grid((T + 7) / 8);
   cudaStream_t s = as_stream(stream);
-  if (keys <= 1)
-    moe::route_topk_kernel<1><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
-  else if (keys <= 2)
-    moe::route_topk_kernel<2><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
-  else if (keys <= 4)
-    moe::route_topk_kernel<4><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
-  else if (keys <= 8)
-    moe::route_topk_kernel<8><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
-  else
-    moe::route_topk_kernel<16><<<grid, block, 0, s>>>(logits, T, E, k, renormalize, topk_idx, topk_w);
-  MOE_CUDA_TRY(cudaGetLastError());
+  auto kern = keys <= 1 ? moe::route_topk_kernel<1>
+            : keys <= 2 ? moe::route_topk_kernel<2>
+            : keys <= 4 ? moe::route_topk_kernel<4>
+            : keys <= 8 ? moe::route_topk_kernel<8>
+                        : moe::route_topk_kernel<16>;
+  MOE_CUDA_TRY(launch_pdl(kern, grid, block, 0, s, logits, T, E, k, renormalize, topk_idx, topk_w));
   return ok();
 }
 
@@ -247,19 +267,17 @@ int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int
                                       (int)moe::permute_smem_bytes(512)));
     attr_set = true;
   }
-  moe::permute_index_kernel<<<1, moe::kPermuteThreads, smem, s>>>(topk_idx, T, E, k, expert_offsets,
-                                                                  perm_token, dest_row);
-  MOE_CUDA_TRY(cudaGetLastError());
+  MOE_CUDA_TRY(launch_pdl(moe::permute_index_kernel, dim3(1), dim3(moe::kPermuteThreads), smem, s,
+                          topk_idx, T, E, k, expert_offsets, perm_token, dest_row));
   const int vec = H / 8;
   const long long nvec = (long long)T * k * vec;
   int dev = 0;
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   const long long cap = (long long)num_sms(dev) * 8;
   const int blocks = (int)std::max(1LL, std::min(cap, (nvec + 255) / 256));
-  moe::gather_rows_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), perm_token,
-                                                  expert_offsets, E, vec,
-                                                  static_cast<uint4*>(x_perm));
-  MOE_CUDA_TRY(cudaGetLastError());
+  MOE_CUDA_TRY(launch_pdl(moe::gather_rows_kernel, dim3(blocks), dim3(256), 0, s,
+                          static_cast<const uint4*>(x), perm_token, expert_offsets, E, vec,
+                          static_cast<uint4*>(x_perm)));
   return ok();
 }
 
@@ -267,13 +285,32 @@ int moe_ffn_workspace_bytes(moe_layer_t L, int rows, size_t* bytes) {
   MOE_CHECK(L != nullptr && bytes != nullptr, MOE_ERR_INVALID_ARG, "null argument");
   MOE_CHECK(rows >= 0, MOE_ERR_INVALID_ARG, "rows=%d < 0", rows);
   const size_t h = ((size_t)rows * L->I * 2 + 255) / 256 * 256;
-  *bytes = h + 256;  // h [rows][I] bf16, then the scheduler's counters
+  *bytes = h + kFfnCounterBytes;  // h [rows][I] bf16, then the scheduler's counters
   return ok();
+}
+
+namespace {
+int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_offsets, int rows,
+                     void* y_perm, void* workspace, size_t workspace_bytes, void* stream,
+                     bool zero_counters);
 }
 
 int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expert_offsets,
                           int rows, void* y_perm, void* workspace, size_t workspace_bytes,
                           void* stream) {
+  return grouped_ffn_impl(L, x_perm, expert_offsets, rows, y_perm, workspace, workspace_bytes,
+                          stream, true);
+}
+
+}  // extern "C"
+
+namespace {
+// zero_counters = false: the caller has already zeroed the scheduler counters
+// on the stream (moe_layer_forward does so first, so that no memset node sits
+// between the layer's kernels).
+int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_offsets, int rows,
+                     void* y_perm, void* workspace, size_t workspace_bytes, void* stream,
+                     bool zero_counters) {
   using namespace moe::ffn;
   MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
   MOE_CHECK(rows >= 0, MOE_ERR_INVALID_ARG, "rows=%d < 0", rows);
@@ -296,8 +333,8 @@ int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expe
   MOE_CHECK(grid > 0, MOE_ERR_CUDA, "cannot query the SM count");
 
   auto* h = static_cast<__nv_bfloat16*>(workspace);
-  int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + need - 256);
-  MOE_CUDA_TRY(cudaMemsetAsync(counters, 0, 2 * sizeof(int), s));
+  int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + need - kFfnCounterBytes);
+  if (zero_counters) MOE_CUDA_TRY(cudaMemsetAsync(counters, 0, ffn_counter_bytes(L->E), s));
 
   // Every expert holds at most T = rows / k rows.  Small groups (decode) use the
   // weights-as-M orientation with a deep pipeline sized for the largest group.
@@ -305,7 +342,7 @@ int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expe
   const bool swap = T <= 128;
   const int xbox = swap ? 16 : 128;
   const int xrows = swap ? std::max(16, (std::min(T, 128) + 15) / 16 * 16) : 128;
-  const int nq = swap ? 6 : 4;
+  const int nq = 4;
   int ns = kMaxNS;
   while (ns > 2 && (int)smem_map(swap, ns, nq, xrows).total > kSmemLimit) --ns;
   const int smem = (int)smem_map(swap, ns, nq, xrows).total;
@@ -319,36 +356,30 @@ int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expe
                  CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != MOE_OK) return rc;
 
-  Params pg{L->d_descs, L->d_prec, expert_offsets, h, counters, L->E, L->H, L->I, L->H, L->I,
-            swap ? L->I / 64 : L->I / 128, xbox, xrows, ns, nq};
-  Params pd{L->d_descs, L->d_prec, expert_offsets, static_cast<__nv_bfloat16*>(y_perm),
-            counters + 1, L->E, L->H, L->I, L->I, L->H, swap ? L->H / 128 : (L->H + 255) / 256,
-            xbox, xrows, ns, nq};
+  Params prm{L->d_descs, L->d_prec, expert_offsets, h, static_cast<__nv_bfloat16*>(y_perm),
+             counters, counters + 16, L->E, L->H, L->I,
+             swap ? L->I / 64 : L->I / 128, swap ? L->H / 128 : (L->H + 255) / 256,
+             xbox, xrows, ns, nq};
 
   static bool attr_set = false;
   if (!attr_set) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<true, true>,
+    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<false, true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<true, false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<false, false>,
+    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<false>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     attr_set = true;
   }
-  if (swap) {
-    grouped_ffn_kernel<true, true><<<grid, kThreads, smem, s>>>(tm_x, pg);
-    MOE_CUDA_TRY(cudaGetLastError());
-    grouped_ffn_kernel<false, true><<<grid, kThreads, smem, s>>>(tm_h, pd);
-  } else {
-    grouped_ffn_kernel<true, false><<<grid, kThreads, smem, s>>>(tm_x, pg);
-    MOE_CUDA_TRY(cudaGetLastError());
-    grouped_ffn_kernel<false, false><<<grid, kThreads, smem, s>>>(tm_h, pd);
-  }
-  MOE_CUDA_TRY(cudaGetLastError());
+  if (swap)
+    MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<true>, dim3(grid), dim3(kThreads), smem, s, tm_x,
+                            tm_h, prm));
+  else
+    MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<false>, dim3(grid), dim3(kThreads), smem, s, tm_x,
+                            tm_h, prm));
   return ok();
 }
+}  // namespace
+
+extern "C" {
 
 int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w, int T, int k,
                 int H, void* out, void* stream) {
@@ -362,9 +393,9 @@ int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w
   const int vec = H / 8;
   const dim3 block(std::min(256, ((vec + 31) / 32) * 32));
   const dim3 grid(T, (vec + block.x - 1) / block.x);
-  moe::combine_kernel<<<grid, block, 0, as_stream(stream)>>>(
-      static_cast<const uint4*>(y_perm), dest_row, topk_w, k, vec, static_cast<uint4*>(out));
-  MOE_CUDA_TRY(cudaGetLastError());
+  MOE_CUDA_TRY(launch_pdl(moe::combine_kernel, grid, block, 0, as_stream(stream),
+                          static_cast<const uint4*>(y_perm), dest_row, topk_w, k, vec,
+                          static_cast<uint4*>(out)));
   return ok();
 }
 
@@ -373,13 +404,21 @@ int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, 
                       int32_t* perm_token, int32_t* dest_row, void* x_perm, void* y_perm,
                       void* workspace, size_t workspace_bytes, void* out, void* stream) {
   MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  if (T > 0) {  // the FFN's scheduler counters, zeroed ahead of the layer's kernels
+    size_t need = 0;
+    moe_ffn_workspace_bytes(L, T * L->k, &need);
+    MOE_CHECK(workspace != nullptr && workspace_bytes >= need, MOE_ERR_INVALID_ARG,
+              "workspace %zu B < %zu B needed", workspace_bytes, need);
+    MOE_CUDA_TRY(cudaMemsetAsync(static_cast<uint8_t*>(workspace) + need - kFfnCounterBytes, 0,
+                                 ffn_counter_bytes(L->E), as_stream(stream)));
+  }
   int rc = moe_route_topk(logits, T, L->E, L->k, renormalize, topk_idx, topk_w, stream);
   if (rc != MOE_OK) return rc;
   rc = moe_permute(topk_idx, x, T, L->E, L->k, L->H, expert_offsets, perm_token, dest_row, x_perm,
                    stream);
   if (rc != MOE_OK) return rc;
-  rc = moe_grouped_ffn_mixed(L, x_perm, expert_offsets, T * L->k, y_perm, workspace,
-                             workspace_bytes, stream);
+  rc = grouped_ffn_impl(L, x_perm, expert_offsets, T * L->k, y_perm, workspace, workspace_bytes,
+                        stream, false);
   if (rc != MOE_OK) return rc;
   return moe_combine(y_perm, dest_row, topk_w, T, L->k, L->H, out, stream);
 }

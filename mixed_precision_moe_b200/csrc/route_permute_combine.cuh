@@ -34,6 +34,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
                                                          int E, int k, int renormalize,
                                                          int32_t* __restrict__ topk_idx,
                                                          float* __restrict__ topk_w) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -129,6 +131,8 @@ __global__ void __launch_bounds__(kPermuteThreads, 1)
   uint32_t* mask = reinterpret_cast<uint32_t*>(psm + kPermuteWarps * E);  // [warps][E]
   int32_t* tot = psm + 2 * kPermuteWarps * E;                   // [E]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_launch_dependents();
+  pdl_wait();
 
   for (int i = tid; i < 2 * kPermuteWarps * E; i += blockDim.x) psm[i] = 0;
   __syncthreads();
@@ -246,6 +250,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           const int32_t* __restrict__ offsets,
                                                           int E, int vec_per_row,
                                                           uint4* __restrict__ x_perm) {
+  pdl_launch_dependents();
+  pdl_wait();
   const size_t n = (size_t)offsets[E] * vec_per_row;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -271,6 +277,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
                                                       const int32_t* __restrict__ dest_row,
                                                       const float* __restrict__ topk_w, int k,
                                                       int vec_per_row, uint4* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int t = blockIdx.x;
   const int c = blockIdx.y * blockDim.x + threadIdx.x;
   if (c >= vec_per_row) return;
