@@ -158,6 +158,31 @@ int moe_grouped_ffn_mixed(moe_layer_t layer, const void* x_perm,
                           const int32_t* expert_offsets, int rows, void* y_perm,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Allocation-free variant of moe_grouped_ffn_mixed (no counterpart on the
+ * pages; it is an interface convenience).  Some callers cannot hand the library
+ * a workspace: code running inside another framework's operator that has no
+ * handle on that framework's allocator, or a latency-critical loop that must not
+ * call cudaMalloc (which may synchronise the device and take milliseconds).
+ * This entry point uses a fixed scratch array that the library keeps in device
+ * memory instead (moe_ffn_noalloc_max_bytes() bytes, 8 MiB, held on every GPU
+ * that loads the library until the process exits) and allocates nothing.
+ *   Same arguments and results as moe_grouped_ffn_mixed, minus the workspace.
+ *   Limit: moe_ffn_workspace_bytes(rows) must not exceed the scratch size, i.e.
+ *   rows * I * 2 + 4096 <= 8 MiB; larger calls fail with MOE_ERR_UNSUPPORTED.
+ *   The first call on a device looks up the scratch's device address (a
+ *   cudaGetSymbolAddress with that device current); make that first call
+ *   before any stream capture.
+ *   All calls on a device share the one scratch array, which keeps the last
+ *   call's contents (the call zeroes the counters it needs): calls that
+ *   overlap on the GPU (different streams, or several layers in flight) race
+ *   and must not be issued. */
+int moe_grouped_ffn_mixed_noalloc(moe_layer_t layer, const void* x_perm,
+                                  const int32_t* expert_offsets, int rows, void* y_perm,
+                                  void* stream);
+
+/* Size in bytes of the scratch array behind moe_grouped_ffn_mixed_noalloc. */
+int moe_ffn_noalloc_max_bytes(size_t* bytes);
+
 /* Weighted combine back to token order (ExactMoE Section 3.4; weights are not
  * renormalised): out[t] = sum_j topk_w[t][j] * y_perm[dest_row[t][j]] in fp32,
  * j in order 0..k-1, pairs with dest_row < 0 skipped, one rounding to bf16.

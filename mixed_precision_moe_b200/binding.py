@@ -33,6 +33,8 @@ SIGNATURES = {
     "moe_permute": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_ffn_workspace_bytes": (_I, [_P, _I, C.POINTER(_S)]),
     "moe_grouped_ffn_mixed": (_I, [_P, _P, _P, _I, _P, _P, _S, _P]),
+    "moe_grouped_ffn_mixed_noalloc": (_I, [_P, _P, _P, _I, _P, _P]),
+    "moe_ffn_noalloc_max_bytes": (_I, [C.POINTER(_S)]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_layer_forward": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _P]),
     "moe_quantize_weights": (_I, [_P, _I, _I, _I, _P, _P, _P]),
@@ -140,6 +142,25 @@ def moe_grouped_ffn_mixed(layer, x_perm, expert_offsets, y_perm=None, workspace=
                                        _ptr(y_perm), _ptr(workspace), workspace.numel(),
                                        _stream(stream)))
     return y_perm
+
+
+def moe_grouped_ffn_mixed_noalloc(layer, x_perm, expert_offsets, y_perm=None, stream=None):
+    """moe_grouped_ffn_mixed with the library's built-in scratch (no workspace);
+    see include/moe.h for the size limit and the no-overlap rule."""
+    _need(x_perm, torch.bfloat16, "x_perm")
+    _need(expert_offsets, torch.int32, "expert_offsets")
+    rows = x_perm.shape[0]
+    if y_perm is None:
+        y_perm = torch.empty((rows, layer.H), dtype=torch.bfloat16, device=x_perm.device)
+    _check(lib().moe_grouped_ffn_mixed_noalloc(layer.handle, _ptr(x_perm), _ptr(expert_offsets),
+                                               rows, _ptr(y_perm), _stream(stream)))
+    return y_perm
+
+
+def moe_ffn_noalloc_max_bytes() -> int:
+    n = C.c_size_t(0)
+    _check(lib().moe_ffn_noalloc_max_bytes(C.byref(n)))
+    return n.value
 
 
 def moe_combine(y_perm, dest_row, topk_w, out=None, stream=None):

@@ -379,7 +379,62 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
 }
 }  // namespace
 
+// ------------------------------------------------- allocation-free FFN entry --
+// Scratch for moe_grouped_ffn_mixed_noalloc: h and the scheduler counters live
+// in this file-scope device array instead of a caller workspace.  Every GPU that
+// loads the library holds it until the process exits.  In host code the name
+// g_ffn_scratch is only a host-side stand-in, so the device address is looked up
+// with cudaGetSymbolAddress, once per device, with that device current.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+__device__ __align__(256) uint8_t g_ffn_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  MOE_CHECK(dev >= 0 && dev < kMaxDevices, MOE_ERR_UNSUPPORTED, "device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_ffn_scratch);
+    MOE_CHECK(e == cudaSuccess && ptr != nullptr, MOE_ERR_CUDA,
+              "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
 extern "C" {
+
+int moe_grouped_ffn_mixed_noalloc(moe_layer_t L, const void* x_perm, const int32_t* expert_offsets,
+                                  int rows, void* y_perm, void* stream) {
+  MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  MOE_CHECK(rows >= 0, MOE_ERR_INVALID_ARG, "rows=%d < 0", rows);
+  if (rows == 0) return ok();
+  size_t need = 0;
+  moe_ffn_workspace_bytes(L, rows, &need);
+  MOE_CHECK(need <= kNoAllocScratchBytes, MOE_ERR_UNSUPPORTED,
+            "rows=%d needs %zu B of scratch; the built-in scratch holds %zu B "
+            "(rows * I * 2 + %zu); use moe_grouped_ffn_mixed with a workspace instead",
+            rows, need, kNoAllocScratchBytes, kFfnCounterBytes);
+  void* scratch = nullptr;
+  int rc = noalloc_scratch(&scratch);
+  if (rc != MOE_OK) return rc;
+  // The counters at the end of the scratch are zeroed on the stream by the call.
+  return grouped_ffn_impl(L, x_perm, expert_offsets, rows, y_perm, scratch, need, stream, true);
+}
+
+int moe_ffn_noalloc_max_bytes(size_t* bytes) {
+  MOE_CHECK(bytes != nullptr, MOE_ERR_INVALID_ARG, "bytes is null");
+  *bytes = kNoAllocScratchBytes;
+  return ok();
+}
 
 int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w, int T, int k,
                 int H, void* out, void* stream) {
