@@ -12,13 +12,15 @@
 // 3.1: the dequantised values define the operations; no FP16 expert is
 // materialised).
 //
-// Design (one persistent CTA per SM, 15 warps):
-//   warp 0       scheduler + TMA producer: takes work units from a global
-//                counter -- every gate/up unit, then every down unit, each in
-//                descending time per unit (INT4/INT8 experts before BF16) --
-//                and streams X tiles and BF16 weight tiles with TMA.  A down
-//                unit first waits (bounded) until all gate/up epilogues of its
+// Design (one persistent CTA per SM, 16 warps):
+//   warp 15      scheduler: takes work units from a global counter -- every
+//                gate/up unit, then every down unit, each in descending time
+//                per unit (INT4/INT8 experts before BF16) -- decodes them and
+//                publishes them to the other roles; before publishing a down
+//                unit it waits (bounded) until all gate/up epilogues of its
 //                expert have published their h rows.
+//   warp 0       TMA producer: streams X tiles and BF16 weight boxes into the
+//                operand ring (one copy per 128 weight rows).
 //   warp 14      code producer: streams INT8/INT4 codes and their fp16 scales
 //                into a staging ring, running ahead of the operand stages.
 //   warp 1       TMEM owner + MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16
@@ -29,14 +31,15 @@
 //   warps 4-7    epilogue: tcgen05.ld, SwiGLU or copy, bf16 stores; gate/up
 //                epilogues publish their rows with a release counter.
 // A work unit is (projection, expert, block of weight rows, tile of rows of
-// that expert).  Weight rows travel in 64-row TMA boxes; for gate/up a unit
-// holds matching gate and up boxes so one epilogue sees g and u of the same
-// feature.  Running both projections in one launch needs one prologue instead
-// of two, and down units fill the tail of the gate/up phase.
+// that expert).  Weight rows travel in 128-row TMA boxes; a gate/up box holds
+// 64 gate rows and the same 64 up rows (a 3-D view of W13), so one epilogue
+// sees g and u of the same feature.  Running both projections in one launch
+// needs one prologue instead of two, and down units fill the tail of the
+// gate/up phase.
 //
 // Two MMA orientations (the host picks one per launch from T = rows / k):
 //   tile mode (large groups, prefill): A = 128 token rows, B = 256 weight rows
-//     (128 gate + 128 up, or 256 down rows), D = 128 x 256 fp32; TMEM lane =
+//     (two gate/up boxes, or 256 down rows), D = 128 x 256 fp32; TMEM lane =
 //     token row.
 //   swap mode (small groups, decode): A = 128 weight rows (64 gate + 64 up, or
 //     128 down rows), B = the group's rows padded to 16, D = 128 x N; lane =
@@ -50,20 +53,20 @@
 namespace moe {
 namespace ffn {
 
-constexpr int kThreads = 480;
-constexpr int kMaxNS = 8;          // operand stages (64 K-elements each)
+constexpr int kThreads = 512;
+constexpr int kMaxNS = 12;         // operand stages (64 K-elements each)
 constexpr int kMaxNQ = 8;          // staging slots for packed weights
 constexpr int kUR = 4;             // work-unit ring depth
 constexpr int kMaxE = 512;
-constexpr int kBoxRows = 64;       // weight rows per TMA box
+constexpr int kBoxRows = 128;      // weight rows per TMA box (gate/up: 64 gate + 64 up)
 constexpr int kDequantWarps = 8;   // warps 2, 3, 8 .. 13
 constexpr int kDequantThreads = 32 * kDequantWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 232448; // dynamic shared memory per block on sm_100
 
 struct alignas(64) ExpertDesc {
-  CUtensorMap tm_w13;  // codes/values of [2I][H]; box 64 rows x (64 bf16 | 64 B)
-  CUtensorMap tm_w2;   // codes/values of [H][I]
+  CUtensorMap tm_w13;  // codes/values of [2I][H] as [2][I][H]; box 2 x 64 rows x (64 bf16 | 64 B)
+  CUtensorMap tm_w2;   // codes/values of [H][I]; box 128 rows x (64 bf16 | 64 B)
   const __half* s13;   // [H/128][2I]
   const __half* s2;    // [I/128][H]
   int prec;            // MOE_BF16 / MOE_INT8 / MOE_INT4, -1 when unset
@@ -72,7 +75,7 @@ struct alignas(64) ExpertDesc {
 static_assert(sizeof(ExpertDesc) == 320, "descriptor layout");
 
 struct Unit {
-  int e, prec, wrow0, nbox;  // expert, precision, first weight row, 64-row boxes
+  int e, prec, wrow0, nbox;  // expert, precision, first weight row (of each half), 128-row boxes
   int row0, nrows;           // rows of the token tile
   int flags;                 // kUnitValid | kUnitGateUp
   int need;                  // down unit: gate/up epilogue arrivals to wait for
@@ -99,6 +102,8 @@ struct Params {
   int xbox_rows;           // rows per X tensor-map box
   int xrows;               // rows of an X stage = rows of a token tile (multiple of 16, <= 128)
   int ns, nq;              // ring depths
+  int acc_stride;          // TMEM columns per accumulator buffer
+  int a_col;               // swap mode: TMEM column of the first A stage (32 columns each)
 };
 
 // Shared-memory map (byte offsets from the 1024-aligned base).
@@ -107,7 +112,9 @@ struct SmemMap {
   uint32_t wstage, xstage, qslot, qscale;
 };
 
-__host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows) {
+constexpr int kNumBarriers = 96;
+
+__host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows, int E) {
   SmemMap m;
   const uint32_t wrows = swap ? 128 : 256;
   m.wstage = wrows * 128;
@@ -127,13 +134,13 @@ __host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows
   off += swap ? 64u * xrows * 4u : 0u;
   off = (off + 15) & ~15u;
   m.bar = off;
-  off += 64 * 8;
+  off += kNumBarriers * 8;
   m.units = off;
   off += kUR * sizeof(Unit);
   m.misc = off;
   off += 64;
   m.entries = off;
-  off += kMaxE * sizeof(Entry) + kMaxE * sizeof(int);  // entries, then first down unit
+  off += E * sizeof(Entry) + E * sizeof(int);  // entries, then first down unit
   m.total = off + 1024;  // slack to align the dynamic shared-memory base
   return m;
 }
@@ -141,8 +148,8 @@ __host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows
 struct Smem {
   uint8_t *w_st, *x_st, *q_st, *q_sc;
   float* xbuf;
-  uint64_t *full, *wfull, *empty, *qfull, *qempty, *accfull, *accempty, *ufull, *uempty;
-  uint64_t *mmadone, *xfull, *xempty;
+  uint64_t *full, *wfull, *empty, *wfree, *qfull, *qempty, *accfull, *accempty, *ufull, *uempty;
+  uint64_t *mmadone, *xfull, *xempty, *go;
   Unit* units;
   uint32_t* tmem_slot;
   int* abort_flag;
@@ -155,7 +162,7 @@ struct Smem {
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* raw, const Params& p, bool swap) {
-  const SmemMap m = smem_map(swap, p.ns, p.nq, p.xrows);
+  const SmemMap m = smem_map(swap, p.ns, p.nq, p.xrows, p.E);
   uint8_t* b = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) &
                                           ~uintptr_t(1023));
   Smem s;
@@ -168,7 +175,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const Params& p, bool swap) 
   s.full = bar;
   s.wfull = s.full + kMaxNS;
   s.empty = s.wfull + kMaxNS;
-  s.qfull = s.empty + kMaxNS;
+  s.wfree = s.empty + kMaxNS;
+  s.qfull = s.wfree + kMaxNS;
   s.qempty = s.qfull + kMaxNQ;
   s.accfull = s.qempty + kMaxNQ;
   s.accempty = s.accfull + 2;
@@ -177,6 +185,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const Params& p, bool swap) 
   s.mmadone = s.uempty + kUR;
   s.xfull = s.mmadone + 1;
   s.xempty = s.xfull + 1;
+  s.go = s.xempty + 1;
   s.units = reinterpret_cast<Unit*>(b + m.units);
   s.tmem_slot = reinterpret_cast<uint32_t*>(b + m.misc);
   s.abort_flag = reinterpret_cast<int*>(b + m.misc + 4);
@@ -184,7 +193,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const Params& p, bool swap) 
   s.n_units = reinterpret_cast<int*>(b + m.misc + 12);
   s.n_units_gu = reinterpret_cast<int*>(b + m.misc + 16);
   s.entries = reinterpret_cast<Entry*>(b + m.entries);
-  s.ub_dn = reinterpret_cast<int*>(b + m.entries + kMaxE * sizeof(Entry));
+  s.ub_dn = reinterpret_cast<int*>(b + m.entries + p.E * sizeof(Entry));
   s.wstage = m.wstage;
   s.xstage = m.xstage;
   s.qslot = m.qslot;
@@ -305,12 +314,12 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
   un.prec = en.e_prec >> 16;
   un.row0 = en.row0 + tt * p.xrows;
   un.nrows = min(p.xrows, en.nrows - tt * p.xrows);
-  if (gu) {  // gate rows [wrow0, wrow0 + rows/2), up rows I + the same
+  if (gu) {  // gate rows [wrow0, wrow0 + 64 nbox), up rows I + the same
     un.wrow0 = wb * (kSwap ? 64 : 128);
-    un.nbox = kSwap ? 2 : 4;
+    un.nbox = kSwap ? 1 : 2;
   } else {
     un.wrow0 = wb * (kSwap ? 128 : 256);
-    un.nbox = min(kSwap ? 2 : 4, (p.H - un.wrow0) / kBoxRows);
+    un.nbox = min(kSwap ? 1 : 2, (p.H - un.wrow0) / kBoxRows);
   }
   un.flags = kUnitValid | (gu ? kUnitGateUp : 0);
   un.need = 4 * tiles_of(en.nrows, p) * p.nwb_gu;  // 4 epilogue warps per gate/up unit
@@ -319,11 +328,31 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
 
 __device__ __forceinline__ bool unit_gu(const Unit& un) { return (un.flags & kUnitGateUp) != 0; }
 
-// First weight row of 64-row box b of a unit.
-__device__ __forceinline__ int box_row(const Params& p, const Unit& un, int b) {
-  if (!unit_gu(un)) return un.wrow0 + kBoxRows * b;
-  const int half = un.nbox >> 1;  // boxes [0, half) gate, [half, nbox) up
-  return b < half ? un.wrow0 + kBoxRows * b : p.I + un.wrow0 + kBoxRows * (b - half);
+// TMA copy of 128-row box b of a unit's weights (values or codes) at K-column
+// kc: gate/up -> gate rows wrow0 + 64 b .. + 63 followed by the same up rows
+// (one copy through the [2][I][K] map); down -> rows wrow0 + 128 b .. + 127.
+__device__ __forceinline__ void load_weight_box(void* dst, const CUtensorMap* tw, const Unit& un,
+                                                int b, int kc, uint64_t* bar) {
+  if (un.flags & kUnitGateUp)
+    tma_load_3d(dst, tw, kc, un.wrow0 + (kBoxRows / 2) * b, 0, bar);
+  else
+    tma_load_2d(dst, tw, kc, un.wrow0 + kBoxRows * b, bar);
+}
+
+// Bulk copies of the fp16 scales of box b for K-group g, in the box's row
+// order (group-major scale arrays: the scales of consecutive rows are
+// contiguous).
+__device__ __forceinline__ void load_scale_box(void* dst, const Params& p, const ExpertDesc* d,
+                                               const Unit& un, int b, int g, uint64_t* bar) {
+  if (un.flags & kUnitGateUp) {
+    const __half* sc = d->s13 + (size_t)g * (2 * p.I) + un.wrow0 + (kBoxRows / 2) * b;
+    constexpr uint32_t kHalfBytes = (kBoxRows / 2) * sizeof(__half);
+    bulk_load(dst, sc, kHalfBytes, bar);                                          // gate rows
+    bulk_load(static_cast<uint8_t*>(dst) + kHalfBytes, sc + p.I, kHalfBytes, bar);  // up rows
+  } else {
+    bulk_load(dst, d->s2 + (size_t)g * p.H + un.wrow0 + kBoxRows * b, kBoxRows * sizeof(__half),
+              bar);
+  }
 }
 
 // Reduction length of the unit's projection in 64-element k-blocks.
@@ -345,9 +374,10 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Down unit: wait until every gate/up epilogue warp of the expert has
-// published its h rows (bounded), then order those generic-proxy writes before
-// this thread's TMA (async-proxy) reads.
+// Down unit: wait (bounded) until every gate/up epilogue warp of the expert
+// has published its h rows.  The acquire makes those writes visible to this
+// CTA; the thread that then reads h with TMA orders them before its
+// async-proxy reads with fence.proxy.async.global.
 __device__ __forceinline__ bool wait_gate_up(const Params& p, const Unit& un,
                                              volatile int* abort_flag) {
   const int* cnt = p.done + un.e;
@@ -357,11 +387,57 @@ __device__ __forceinline__ bool wait_gate_up(const Params& p, const Unit& un,
     if (clock64() - t0 > kWaitLimitCycles) return false;
     __nanosleep(128);
   }
-  fence_proxy_async_global();
   return true;
 }
 
+// --------------------------------------------------------------- scheduler --
+// Takes units from the global counter, decodes them, prefetches the weight
+// tensor map and, for a down unit, waits for its gate/up rows, then publishes
+// the unit to every role through the unit ring.  It reserves unit n + 1 only
+// when the producer reaches the reserve point of unit n (the `go` barrier), a
+// few k-blocks before unit n's last copies: every global round trip of a unit
+// switch happens here, off the producer's path, while the late reservation
+// keeps the dynamic balance of the tail.
+template <bool kSwap>
+__device__ void scheduler(const Params& p, const Smem& s) {
+  volatile int* abort_flag = s.abort_flag;
+  const int total = *s.n_units;
+  uint32_t us = 0, uph = 0, gph = 0;
+  bool ok = true;
+  for (bool first = true;; first = false) {
+    if (!first) {
+      if (!mbar_wait(s.go, gph, abort_flag)) {
+        ok = false;
+        break;
+      }
+      gph ^= 1u;
+    }
+    const int u = atomicAdd(p.counter, 1);
+    Unit un = Unit{0, 0, 0, 0, 0, 0, 0, 0};
+    if (u < total) {
+      un = decode_unit<kSwap>(p, s, u);
+      const ExpertDesc* d = p.descs + un.e;
+      prefetch_tmap(unit_gu(un) ? &d->tm_w13 : &d->tm_w2);
+      if (!unit_gu(un) && !wait_gate_up(p, un, abort_flag)) {
+        ok = false;
+        break;
+      }
+    }
+    if (!mbar_wait(&s.uempty[us], uph ^ 1u, abort_flag)) {
+      ok = false;
+      break;
+    }
+    s.units[us] = un;
+    mbar_arrive(&s.ufull[us]);
+    advance(us, uph, kUR);
+    if (!(un.flags & kUnitValid)) break;
+  }
+  if (!ok) give_up(s);
+}
+
 // ---------------------------------------------------------------- producer --
+// Streams, per k-block, the X tile (one copy) and, for BF16 units, the
+// weight boxes into the operand ring.
 template <bool kSwap>
 __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const Params& p,
                          const Smem& s) {
@@ -369,25 +445,17 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
   const uint32_t ns = p.ns;
   uint32_t st = 0, sph = 0, us = 0, uph = 0;
   uint32_t issued = 0, issued_par = 0;  // drain bookkeeping
-  const int total = *s.n_units;
+  const uint32_t xbytes = (uint32_t)p.xbox_rows * 128;
   bool ok = true;
   prefetch_tmap(tm_x);
   prefetch_tmap(tm_h);
-  int next_u = atomicAdd(p.counter, 1);
   for (;;) {
-    if (!mbar_wait(&s.uempty[us], uph ^ 1u, abort_flag)) {
+    if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
       ok = false;
       break;
     }
-    const int u = next_u;
-    Unit un;
-    if (u < total) {
-      un = decode_unit<kSwap>(p, s, u);
-    } else {
-      un = Unit{0, 0, 0, 0, 0, 0, 0, 0};
-    }
-    s.units[us] = un;
-    mbar_arrive(&s.ufull[us]);
+    const Unit un = s.units[us];
+    mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
 
@@ -395,34 +463,25 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
     const ExpertDesc* d = p.descs + un.e;
     const CUtensorMap* tw = gu ? &d->tm_w13 : &d->tm_w2;
     const CUtensorMap* tx = gu ? tm_x : tm_h;
-    if (un.prec == MOE_BF16) {
-      tmap_acquire(tw);
-      prefetch_tmap(tw);
-    }
-    if (!gu && !wait_gate_up(p, un, abort_flag)) {
-      ok = false;
-      break;
-    }
+    const bool bf16 = un.prec == MOE_BF16;
+    if (bf16) tmap_acquire(tw);
+    if (!gu) fence_proxy_async_global();  // h rows published (scheduler's acquire) -> TMA reads
     const int nkb = unit_nkb(p, un);
-    const int nxb = (un.nrows + p.xbox_rows - 1) / p.xbox_rows;
-    const uint32_t xbytes = (uint32_t)(nxb * p.xbox_rows * 128);
-    const int prefetch_kb = max(0, nkb - (int)ns);  // reserve the next unit near the end
+    const uint32_t bytes = xbytes + (bf16 ? (uint32_t)un.nbox * (kBoxRows * 128) : 0u);
+    const int reserve_kb = max(0, nkb - (int)ns - 4);
     for (int kb = 0; kb < nkb; ++kb) {
-      if (kb == prefetch_kb) next_u = atomicAdd(p.counter, 1);
+      if (kb == reserve_kb) mbar_arrive(s.go);
       if (!mbar_wait(&s.empty[st], sph ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
-      const uint32_t bytes =
-          xbytes + (un.prec == MOE_BF16 ? (uint32_t)un.nbox * (kBoxRows * 128) : 0u);
+      if (!bf16) mbar_arrive(&s.wfree[st]);  // the dequant warps may fill this stage
       mbar_arrive_expect_tx(&s.full[st], bytes);
-      for (int b = 0; b < nxb; ++b)
-        tma_load_2d(s.x_st + st * s.xstage + b * p.xbox_rows * 128, tx, kb * 64,
-                    un.row0 + b * p.xbox_rows, &s.full[st]);
-      if (un.prec == MOE_BF16)
+      tma_load_2d(s.x_st + st * s.xstage, tx, kb * 64, un.row0, &s.full[st]);
+      if (bf16)
         for (int b = 0; b < un.nbox; ++b)
-          tma_load_2d(s.w_st + st * s.wstage + b * (kBoxRows * 128), tw, kb * 64,
-                      box_row(p, un, b), &s.full[st]);
+          load_weight_box(s.w_st + st * s.wstage + b * (kBoxRows * 128), tw, un, b, kb * 64,
+                          &s.full[st]);
       issued |= 1u << st;
       issued_par = (issued_par & ~(1u << st)) | (sph << st);
       advance(st, sph, ns);
@@ -460,8 +519,6 @@ __device__ void code_producer(const Params& p, const Smem& s) {
     const bool gu = unit_gu(un);
     const ExpertDesc* d = p.descs + un.e;
     const CUtensorMap* tw = gu ? &d->tm_w13 : &d->tm_w2;
-    const __half* sc = gu ? d->s13 : d->s2;
-    const int srows = gu ? 2 * p.I : p.H;  // rows of the scale matrix
     tmap_acquire(tw);
     prefetch_tmap(tw);
     const int nkb = unit_nkb(p, un);
@@ -475,10 +532,8 @@ __device__ void code_producer(const Params& p, const Smem& s) {
       const int kc = int4 ? (kb >> 1) * 64 : kb * 64;  // byte column of the codes
       const int g = kb >> 1;                            // K-group of the scales
       for (int b = 0; b < un.nbox; ++b) {
-        const int wr = box_row(p, un, b);
-        tma_load_2d(s.q_st + q * s.qslot + b * (kBoxRows * 64), tw, kc, wr, &s.qfull[q]);
-        bulk_load(s.q_sc + q * s.qscale + b * (kBoxRows * 2), sc + (size_t)g * srows + wr,
-                  kBoxRows * 2, &s.qfull[q]);
+        load_weight_box(s.q_st + q * s.qslot + b * (kBoxRows * 64), tw, un, b, kc, &s.qfull[q]);
+        load_scale_box(s.q_sc + q * s.qscale + b * (kBoxRows * 2), p, d, un, b, g, &s.qfull[q]);
       }
       qissued |= 1u << q;
       qissued_par = (qissued_par & ~(1u << q)) | (qph << q);
@@ -495,15 +550,40 @@ __device__ void code_producer(const Params& p, const Smem& s) {
 
 // -------------------------------------------------------------- MMA issuer --
 // TMEM columns: tile mode uses two 256-column accumulators; swap mode uses two
-// 128-column accumulators (N <= 128) and, from column kATmemCol, one 32-column
-// A stage per operand stage (64 K-elements x 128 rows of dequantised weights).
-constexpr uint32_t kATmemCol = 256;
+// accumulators of acc_stride columns (the power of two >= the token tile, so
+// N <= acc_stride) and, from column a_col = 2 * acc_stride, one 32-column A
+// stage per operand stage (64 K-elements x 128 rows of dequantised weights).
+
+// Four K=16 MMAs over one 64-element k-block.  The operand descriptors are
+// formed once per stage by adding to base descriptors (the start-address field
+// is the low 14 bits, in 16-byte units; +2 per 32-byte K step inside the
+// 128-byte swizzle row), and the sequence is fully unrolled with no branch
+// between the MMAs: in this form the issuing thread keeps the tensor core fed
+// (about 4x cheaper per MMA than computing each descriptor in the loop).
+__device__ __forceinline__ void mma_kblock_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t acc0) {
+  mma_bf16_ss(d, a, b, idesc, acc0);
+  mma_bf16_ss(d, a + 2, b + 2, idesc, 1u);
+  mma_bf16_ss(d, a + 4, b + 4, idesc, 1u);
+  mma_bf16_ss(d, a + 6, b + 6, idesc, 1u);
+}
+
+__device__ __forceinline__ void mma_kblock_ts(uint32_t d, uint32_t a_tmem, uint64_t b,
+                                              uint32_t idesc, uint32_t acc0) {
+  mma_bf16_ts(d, a_tmem, b, idesc, acc0);
+  mma_bf16_ts(d, a_tmem + 8, b + 2, idesc, 1u);
+  mma_bf16_ts(d, a_tmem + 16, b + 4, idesc, 1u);
+  mma_bf16_ts(d, a_tmem + 24, b + 6, idesc, 1u);
+}
 
 template <bool kSwap>
 __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
-  constexpr uint32_t kAccCols = kSwap ? 128 : 256;
+  const uint32_t acc_cols = p.acc_stride, a_tmem0 = tmem + p.a_col;
   volatile int* abort_flag = s.abort_flag;
   const uint32_t ns = p.ns;
+  const uint64_t wdesc0 = smem_desc_sw128(smem_u32(s.w_st));
+  const uint64_t xdesc0 = smem_desc_sw128(smem_u32(s.x_st));
+  const uint32_t wstep = s.wstage >> 4, xstep = s.xstage >> 4;
   uint32_t st = 0, sph = 0, us = 0, uph = 0, abuf = 0;
   uint32_t aph[2] = {0, 0};
   uint32_t wph = 0;  // wfull phase bit per stage: it only advances on INT8/INT4 units
@@ -523,7 +603,7 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
       break;
     }
     tc_fence_after();
-    const uint32_t d_tmem = tmem + abuf * kAccCols;
+    const uint32_t d_tmem = tmem + abuf * acc_cols;
     const int n = kSwap ? max(16, (un.nrows + 15) & ~15) : un.nbox * kBoxRows;
     const uint32_t idesc = idesc_bf16_f32(128, n);
     const bool quant = un.prec != MOE_BF16;
@@ -536,21 +616,14 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
       }
       if (quant) wph ^= 1u << st;
       tc_fence_after();
-      const uint32_t xa = smem_u32(s.x_st + st * s.xstage);
-      const uint32_t wa = smem_u32(s.w_st + st * s.wstage);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t acc = (kb | kk) != 0;
-        if (a_in_tmem)
-          mma_bf16_ts(d_tmem, tmem + kATmemCol + st * 32 + kk * 8, smem_desc_sw128(xa + kk * 32),
-                      idesc, acc);
-        else if (kSwap)
-          mma_bf16_ss(d_tmem, smem_desc_sw128(wa + kk * 32), smem_desc_sw128(xa + kk * 32), idesc,
-                      acc);
-        else
-          mma_bf16_ss(d_tmem, smem_desc_sw128(xa + kk * 32), smem_desc_sw128(wa + kk * 32), idesc,
-                      acc);
-      }
+      const uint64_t xd = xdesc0 + st * xstep, wd = wdesc0 + st * wstep;
+      const uint32_t acc0 = kb != 0;
+      if (a_in_tmem)
+        mma_kblock_ts(d_tmem, a_tmem0 + st * 32, xd, idesc, acc0);
+      else if (kSwap)
+        mma_kblock_ss(d_tmem, wd, xd, idesc, acc0);
+      else
+        mma_kblock_ss(d_tmem, xd, wd, idesc, acc0);
       mma_commit(&s.empty[st]);
       advance(st, sph, ns);
     }
@@ -566,6 +639,16 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
 }
 
 // ----------------------------------------------------------------- dequant --
+// The dequant warps take part only in INT8/INT4 positions of the operand ring
+// and pass over BF16 units at once, so they may be any number of ring
+// revolutions away from the producer and the MMA; a parity wait on a barrier
+// that completes at every position (empty) could then match the wrong phase.
+// They wait instead on wfree[st], which the producer arrives on (after its own
+// empty wait, i.e. once the previous use of the stage is complete) only at
+// INT8/INT4 positions, and count its phases per stage: at most one phase of
+// wfree[st] is ever outstanding, so the parity is exact.
+
+
 // Code -> bf16 dequantisation, exact up to the final rounding.  A code byte u
 // (INT4: the nibble, u = q + 8; INT8: the byte xor 0x80, u = q + 128) becomes
 // the fp32 m = 2^15 + u by placing it in mantissa bits 8..15 of 2^15 (one
@@ -621,9 +704,10 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
   const int quarter = warp & 3;
   const int half = warp >= 10 ? 1 : 0;
   const int r = quarter * 32 + lane;  // weight row of the unit = TMEM lane
-  const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + kATmemCol;
+  const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + p.a_col;
   const uint32_t ns = p.ns, nq = p.nq;
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
+  uint32_t fph = 0;  // wfree phase bit per stage: it only advances on INT8/INT4 positions
   bool ok = true;
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
@@ -643,16 +727,17 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
     const bool int4 = un.prec == MOE_INT4;
     const float off = int4 ? 32776.0f : 32896.0f;  // 2^15 + 8, 2^15 + 128
     for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
-      const uint32_t st0 = st, sph0 = sph;
+      const uint32_t st0 = st;
       advance(st, sph, ns);
-      const uint32_t st1 = st, sph1 = sph;
+      const uint32_t st1 = st;
       if (int4) advance(st, sph, ns);
       if (!mbar_wait(&s.qfull[q], qph, abort_flag) ||
-          !mbar_wait(&s.empty[st0], sph0 ^ 1u, abort_flag) ||
-          (int4 && !mbar_wait(&s.empty[st1], sph1 ^ 1u, abort_flag))) {
+          !mbar_wait(&s.wfree[st0], (fph >> st0) & 1u, abort_flag) ||
+          (int4 && !mbar_wait(&s.wfree[st1], (fph >> st1) & 1u, abort_flag))) {
         ok = false;
         break;
       }
+      fph ^= (1u << st0) | (int4 ? 1u << st1 : 0u);
       tc_fence_after();
       const uint4* src = reinterpret_cast<const uint4*>(s.q_st + q * s.qslot + r * 64 + half * 32);
       const uint4 c0 = src[0], c1 = src[1];
@@ -698,6 +783,7 @@ __device__ void dequant(const Params& p, const Smem& s, int dtid) {
   const int lane = threadIdx.x & 31;
   const uint32_t ns = p.ns, nq = p.nq;
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
+  uint32_t fph = 0;  // wfree phase bit per stage: it only advances on INT8/INT4 positions
   constexpr int kMaxItems = 4;  // 256 rows x 4 items / kDequantThreads
   bool ok = true;
   for (;;) {
@@ -720,16 +806,17 @@ __device__ void dequant(const Params& p, const Smem& s, int dtid) {
     const float off = int4 ? 32776.0f : 32896.0f;  // 2^15 + 8, 2^15 + 128
     const uint32_t flip = int4 ? 0u : 0x80808080u;
     for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
-      const uint32_t st0 = st, sph0 = sph;
+      const uint32_t st0 = st;
       advance(st, sph, ns);
-      const uint32_t st1 = st, sph1 = sph;
+      const uint32_t st1 = st;
       if (int4) advance(st, sph, ns);
       if (!mbar_wait(&s.qfull[q], qph, abort_flag) ||
-          !mbar_wait(&s.empty[st0], sph0 ^ 1u, abort_flag) ||
-          (int4 && !mbar_wait(&s.empty[st1], sph1 ^ 1u, abort_flag))) {
+          !mbar_wait(&s.wfree[st0], (fph >> st0) & 1u, abort_flag) ||
+          (int4 && !mbar_wait(&s.wfree[st1], (fph >> st1) & 1u, abort_flag))) {
         ok = false;
         break;
       }
+      fph ^= (1u << st0) | (int4 ? 1u << st1 : 0u);
       const uint8_t* qs = s.q_st + q * s.qslot;
       const __half* scs = reinterpret_cast<const __half*>(s.q_sc + q * s.qscale);
       const uint32_t w0 = smem_u32(s.w_st + st0 * s.wstage);
@@ -808,7 +895,7 @@ __device__ __forceinline__ void publish_rows(const Params& p, const Unit& un, in
 
 template <bool kSwap>
 __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
-  constexpr uint32_t kAccCols = kSwap ? 128 : 256;
+  const uint32_t acc_cols = p.acc_stride;
   volatile int* abort_flag = s.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
@@ -831,7 +918,7 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
       break;
     }
     tc_fence_after();
-    const uint32_t tb = tmem + ((uint32_t)(quarter * 32) << 16) + ebuf * kAccCols;
+    const uint32_t tb = tmem + ((uint32_t)(quarter * 32) << 16) + ebuf * acc_cols;
     if (kSwap) {
       const int wr = quarter * 32 + lane;  // weight row of the unit (TMEM lane)
       const int n_pad = max(16, (un.nrows + 15) & ~15);
@@ -883,26 +970,32 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
         }
       }
     } else {
+      // D columns follow the weight rows of the stage: gate/up boxes hold 64
+      // gate rows then the same 64 up rows, so column 128 c + j (j < 64) pairs
+      // with 128 c + 64 + j and is feature wrow0 + 64 c + j.
       const int m = quarter * 32 + lane;  // token row inside the tile
       const bool valid = m < un.nrows;
-      __nv_bfloat16* out = gu ? p.h + (size_t)(un.row0 + m) * p.I + un.wrow0
-                              : p.y + (size_t)(un.row0 + m) * p.H + un.wrow0;
-      uint4* dst = reinterpret_cast<uint4*>(out);
-      const int ncols = gu ? 128 : un.nbox * kBoxRows;
-      for (int c0 = 0; c0 < ncols; c0 += 16) {
-        uint32_t a[16], b[16];
-        tmem_ld16(tb + c0, a);
-        if (gu) tmem_ld16(tb + 128 + c0, b);
-        tmem_ld_wait();
-        float f[16];
+      if (quarter * 32 < un.nrows) {      // warps holding no row of the tile skip
+        __nv_bfloat16* out = gu ? p.h + (size_t)(un.row0 + m) * p.I + un.wrow0
+                                : p.y + (size_t)(un.row0 + m) * p.H + un.wrow0;
+        uint4* dst = reinterpret_cast<uint4*>(out);
+        const int ncols = gu ? un.nbox * (kBoxRows / 2) : un.nbox * kBoxRows;
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+          uint32_t a[16], b[16];
+          const uint32_t col = gu ? (c0 / 64) * 128 + (c0 % 64) : c0;
+          tmem_ld16(tb + col, a);
+          if (gu) tmem_ld16(tb + col + 64, b);
+          tmem_ld_wait();
+          float f[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          f[j] = gu ? silu_mul(__uint_as_float(a[j]), __uint_as_float(b[j])) : __uint_as_float(a[j]);
-        if (valid) {
-          dst[c0 / 8] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                   pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-          dst[c0 / 8 + 1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
-                                       pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+          for (int j = 0; j < 16; ++j)
+            f[j] = gu ? silu_mul(__uint_as_float(a[j]), __uint_as_float(b[j])) : __uint_as_float(a[j]);
+          if (valid) {
+            dst[c0 / 8] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+            dst[c0 / 8 + 1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
+                                         pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+          }
         }
       }
     }
@@ -925,28 +1018,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Smem s = carve(ffn_smem_raw, p, kSwap);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  {  // barrier initialisation, one barrier per thread of warps 2 and 3
+  {  // barrier initialisation, one barrier (set) per thread of warps 2 and 3
+    constexpr int kAccInit = kMaxNS + kMaxNQ, kUnitInit = kAccInit + 2;
+    static_assert(kUnitInit + kUR < 64, "barrier initialisation needs more threads");
     const int i = threadIdx.x - 64;
     if (i >= 0 && i < kMaxNS) {
       mbar_init(&s.full[i], 1);                // producer's arrive.expect_tx
       mbar_init(&s.wfull[i], kDequantWarps);   // one arrival per dequant warp
       mbar_init(&s.empty[i], 1);               // tcgen05.commit
+      mbar_init(&s.wfree[i], 1);               // producer, at INT8/INT4 positions
     } else if (i >= kMaxNS && i < kMaxNS + kMaxNQ) {
       mbar_init(&s.qfull[i - kMaxNS], 1);
       mbar_init(&s.qempty[i - kMaxNS], kDequantWarps);
-    } else if (i >= 16 && i < 18) {
-      mbar_init(&s.accfull[i - 16], 1);
-      mbar_init(&s.accempty[i - 16], 4);
-    } else if (i >= 18 && i < 18 + kUR) {
-      mbar_init(&s.ufull[i - 18], 1);
-      mbar_init(&s.uempty[i - 18], 2 + 4 + kDequantWarps);  // MMA, code producer, epilogue, dequant
-    } else if (i == 30) {
+    } else if (i >= kAccInit && i < kAccInit + 2) {
+      mbar_init(&s.accfull[i - kAccInit], 1);
+      mbar_init(&s.accempty[i - kAccInit], 4);
+    } else if (i >= kUnitInit && i < kUnitInit + kUR) {
+      mbar_init(&s.ufull[i - kUnitInit], 1);
+      // producer, MMA, code producer, 4 epilogue warps, dequant warps
+      mbar_init(&s.uempty[i - kUnitInit], 3 + 4 + kDequantWarps);
+    } else if (i == kUnitInit + kUR) {
       mbar_init(s.mmadone, 1);
       mbar_init(s.xfull, 2);   // the two epilogue warps holding the up half
       mbar_init(s.xempty, 2);  // the two epilogue warps holding the gate half
+      mbar_init(s.go, 1);      // producer: reserve the next unit
       *s.abort_flag = 0;
     }
-    if (i >= 0 && i < 32) fence_mbar_init();
+    if (i >= 0 && i < 64) fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(s.tmem_slot, kTmemCols);
@@ -968,6 +1066,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     epilogue<kSwap>(p, s, tmem);
   } else if (warp == 14) {
     if (lane == 0) code_producer(p, s);
+  } else if (warp == 15) {
+    if (lane == 0) scheduler<kSwap>(p, s);
   } else {
     if (kSwap) {
       dequant_tmem(p, s, tmem);

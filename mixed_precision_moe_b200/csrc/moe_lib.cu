@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -88,17 +89,41 @@ int encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int e
   return MOE_OK;
 }
 
-// Tensor map of one expert weight matrix [rows][K] in its storage format:
-// BF16 -> box 64 rows x 64 bf16 (128-byte swizzle, the MMA operand layout);
-// INT8/INT4 -> box 64 rows x 64 bytes of codes (staged, then dequantised).
-int encode_weight(CUtensorMap* m, const void* base, int prec, int rows, int K) {
-  const uint32_t box_rows = moe::ffn::kBoxRows;
-  if (prec == MOE_BF16)
-    return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, box_rows, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-  const int cols = (prec == MOE_INT4) ? K / 2 : K;
-  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, box_rows, 64,
-                   CU_TENSOR_MAP_SWIZZLE_NONE);
+// 3-D map over a row-major [d2][rows][cols] array; box = box_d2 x box_rows x
+// box_cols elements.
+int encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int esize,
+              uint64_t d2, uint64_t rows, uint64_t cols, uint32_t box_d2, uint32_t box_rows,
+              uint32_t box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  MOE_CHECK(fn != nullptr, MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {cols, rows, d2};
+  cuuint64_t strides[2] = {cols * (uint64_t)esize, rows * cols * (uint64_t)esize};
+  cuuint32_t box[3] = {box_cols, box_rows, box_d2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MOE_CHECK(r == CUDA_SUCCESS, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOE_OK;
+}
+
+// Tensor maps of one expert's weights in their storage format.  Every box
+// holds 128 weight rows x 64 K-elements, so one TMA fetches a whole 128-row
+// operand block:
+//   w13 [2I][K] is mapped as [2][I][K] with box 2 x 64 x 64: rows r .. r+63 of
+//     the gate half and the same rows of the up half in one copy;
+//   w2 [H][K] as a 2-D map with box 128 x 64.
+// BF16 values land in the 128-byte-swizzled layout the MMA reads; INT8/INT4
+// codes (64 bytes of a row per box) are staged unswizzled and dequantised.
+int encode_weights(moe::ffn::ExpertDesc* d, const moe_expert_weights* w, int prec, int H, int I) {
+  const bool bf16 = prec == MOE_BF16;
+  const CUtensorMapDataType t = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const int es = bf16 ? 2 : 1;
+  const CUtensorMapSwizzle swz = bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const int cols13 = prec == MOE_INT4 ? H / 2 : H, cols2 = prec == MOE_INT4 ? I / 2 : I;
+  int rc = encode_3d(&d->tm_w13, w->w13, t, es, 2, I, cols13, 2, 64, 64, swz);
+  if (rc != MOE_OK) return rc;
+  return encode_2d(&d->tm_w2, w->w2, t, es, H, cols2, 128, 64, swz);
 }
 
 // Launch with programmatic stream serialization: the kernel may be scheduled
@@ -201,9 +226,7 @@ int moe_set_expert_precision(moe_layer_t L, int expert, moe_precision_t precisio
   }
   moe::ffn::ExpertDesc d;
   memset(&d, 0, sizeof d);
-  int rc = encode_weight(&d.tm_w13, w->w13, prec, 2 * L->I, L->H);
-  if (rc != MOE_OK) return rc;
-  rc = encode_weight(&d.tm_w2, w->w2, prec, L->H, L->I);
+  const int rc = encode_weights(&d, w, prec, L->H, L->I);
   if (rc != MOE_OK) return rc;
   d.s13 = prec == MOE_BF16 ? nullptr : static_cast<const __half*>(w->s13);
   d.s2 = prec == MOE_BF16 ? nullptr : static_cast<const __half*>(w->s2);
@@ -305,6 +328,24 @@ int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expe
 }  // extern "C"
 
 namespace {
+constexpr int kMaxDevices = 64;
+
+// The kernel's dynamic shared-memory limit is a per-device function attribute;
+// it is set once per device.
+int set_ffn_attributes(int dev) {
+  static std::atomic<bool> done[kMaxDevices];
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && done[dev].load()) return MOE_OK;
+  MOE_CUDA_TRY(cudaFuncSetAttribute(moe::ffn::grouped_ffn_kernel<true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    moe::ffn::kSmemLimit));
+  MOE_CUDA_TRY(cudaFuncSetAttribute(moe::ffn::grouped_ffn_kernel<false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    moe::ffn::kSmemLimit));
+  if (cached) done[dev].store(true);
+  return MOE_OK;
+}
+
 // zero_counters = false: the caller has already zeroed the scheduler counters
 // on the stream (moe_layer_forward does so first, so that no memset node sits
 // between the layer's kernels).
@@ -340,12 +381,22 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
   // weights-as-M orientation with a deep pipeline sized for the largest group.
   const int T = (rows + L->k - 1) / L->k;
   const bool swap = T <= 128;
-  const int xbox = swap ? 16 : 128;
   const int xrows = swap ? std::max(16, (std::min(T, 128) + 15) / 16 * 16) : 128;
+  const int xbox = xrows;  // one X copy per stage
   const int nq = 4;
-  int ns = kMaxNS;
-  while (ns > 2 && (int)smem_map(swap, ns, nq, xrows).total > kSmemLimit) --ns;
-  const int smem = (int)smem_map(swap, ns, nq, xrows).total;
+  // TMEM (512 columns): swap mode holds two accumulators of acc_stride columns
+  // (a power of two >= the token tile) and one 32-column A stage per operand
+  // stage; tile mode two 256-column accumulators.
+  int acc_stride = 256;
+  if (swap) {
+    acc_stride = 16;
+    while (acc_stride < xrows) acc_stride *= 2;
+  }
+  const int a_col = swap ? 2 * acc_stride : 0;
+  const int ns_tmem = swap ? ((int)kTmemCols - a_col) / 32 : kMaxNS;
+  int ns = std::min(kMaxNS, ns_tmem);
+  while (ns > 2 && (int)smem_map(swap, ns, nq, xrows, L->E).total > kSmemLimit) --ns;
+  const int smem = (int)smem_map(swap, ns, nq, xrows, L->E).total;
   MOE_CHECK(smem <= kSmemLimit, MOE_ERR_UNSUPPORTED, "shared memory plan does not fit");
 
   CUtensorMap tm_x, tm_h;
@@ -359,16 +410,10 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
   Params prm{L->d_descs, L->d_prec, expert_offsets, h, static_cast<__nv_bfloat16*>(y_perm),
              counters, counters + 16, L->E, L->H, L->I,
              swap ? L->I / 64 : L->I / 128, swap ? L->H / 128 : (L->H + 255) / 256,
-             xbox, xrows, ns, nq};
+             xbox, xrows, ns, nq, acc_stride, a_col};
 
-  static bool attr_set = false;
-  if (!attr_set) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_ffn_kernel<false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-    attr_set = true;
-  }
+  rc = set_ffn_attributes(dev);
+  if (rc != MOE_OK) return rc;
   if (swap)
     MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<true>, dim3(grid), dim3(kThreads), smem, s, tm_x,
                             tm_h, prm));
@@ -389,7 +434,6 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 __device__ __align__(256) uint8_t g_ffn_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
 
