@@ -63,6 +63,7 @@ constexpr int kDequantWarps = 8;   // warps 2, 3, 8 .. 13
 constexpr int kDequantThreads = 32 * kDequantWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 232448; // dynamic shared memory per block on sm_100
+constexpr long long kDrainCycles = 2000000;  // ~1 ms: bound of a wait in the give-up path
 
 struct alignas(64) ExpertDesc {
   CUtensorMap tm_w13;  // codes/values of [2I][H] as [2][I][H]; box 2 x 64 rows x (64 bf16 | 64 B)
@@ -148,7 +149,7 @@ __host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows
 struct Smem {
   uint8_t *w_st, *x_st, *q_st, *q_sc;
   float* xbuf;
-  uint64_t *full, *wfull, *empty, *wfree, *qfull, *qempty, *accfull, *accempty, *ufull, *uempty;
+  uint64_t *full, *empty, *wfree, *qfull, *qempty, *accfull, *accempty, *ufull, *uempty;
   uint64_t *mmadone, *xfull, *xempty, *go;
   Unit* units;
   uint32_t* tmem_slot;
@@ -173,8 +174,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const Params& p, bool swap) 
   s.xbuf = reinterpret_cast<float*>(b + m.xb);
   uint64_t* bar = reinterpret_cast<uint64_t*>(b + m.bar);
   s.full = bar;
-  s.wfull = s.full + kMaxNS;
-  s.empty = s.wfull + kMaxNS;
+  s.empty = s.full + kMaxNS;
   s.wfree = s.empty + kMaxNS;
   s.qfull = s.wfree + kMaxNS;
   s.qempty = s.qfull + kMaxNQ;
@@ -477,6 +477,7 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
       }
       if (!bf16) mbar_arrive(&s.wfree[st]);  // the dequant warps may fill this stage
       mbar_arrive_expect_tx(&s.full[st], bytes);
+      if (bf16) mbar_arrive_n(&s.full[st], kDequantWarps);  // no dequant at this position
       tma_load_2d(s.x_st + st * s.xstage, tx, kb * 64, un.row0, &s.full[st]);
       if (bf16)
         for (int b = 0; b < un.nbox; ++b)
@@ -490,9 +491,12 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
   }
   if (!ok) {
     give_up(s);
-    // Let copies already in flight land before the CTA's shared memory goes away.
+    // Let copies already in flight land before the CTA's shared memory goes
+    // away.  The full barrier of an INT8/INT4 position also counts dequant
+    // arrivals, which may never come once the CTA gives up, so each wait is
+    // cut short after about a millisecond (copies land within microseconds).
     for (uint32_t i = 0; i < ns; ++i)
-      if (issued & (1u << i)) mbar_wait(&s.full[i], (issued_par >> i) & 1u);
+      if (issued & (1u << i)) mbar_wait(&s.full[i], (issued_par >> i) & 1u, nullptr, kDrainCycles);
   }
 }
 
@@ -586,7 +590,6 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
   const uint32_t wstep = s.wstage >> 4, xstep = s.xstage >> 4;
   uint32_t st = 0, sph = 0, us = 0, uph = 0, abuf = 0;
   uint32_t aph[2] = {0, 0};
-  uint32_t wph = 0;  // wfull phase bit per stage: it only advances on INT8/INT4 units
   bool ok = true;
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
@@ -609,12 +612,10 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
     const bool quant = un.prec != MOE_BF16;
     const bool a_in_tmem = kSwap && quant;  // dequantised weights live in TMEM
     for (int kb = 0; kb < nkb; ++kb) {
-      if (!mbar_wait(&s.full[st], sph, abort_flag) ||
-          (quant && !mbar_wait(&s.wfull[st], (wph >> st) & 1u, abort_flag))) {
+      if (!mbar_wait(&s.full[st], sph, abort_flag)) {  // X landed, weights in place
         ok = false;
         break;
       }
-      if (quant) wph ^= 1u << st;
       tc_fence_after();
       const uint64_t xd = xdesc0 + st * xstep, wd = wdesc0 + st * wstep;
       const uint32_t acc0 = kb != 0;
@@ -767,8 +768,8 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {  // one arrival per dequant warp and stage
-        mbar_arrive(&s.wfull[st0]);
-        if (int4) mbar_arrive(&s.wfull[st1]);
+        mbar_arrive(&s.full[st0]);
+        if (int4) mbar_arrive(&s.full[st1]);
         mbar_arrive(&s.qempty[q]);
       }
       advance(q, qph, nq);
@@ -869,8 +870,8 @@ __device__ void dequant(const Params& p, const Smem& s, int dtid) {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {  // one arrival per dequant warp and stage
-        mbar_arrive(&s.wfull[st0]);
-        if (int4) mbar_arrive(&s.wfull[st1]);
+        mbar_arrive(&s.full[st0]);
+        if (int4) mbar_arrive(&s.full[st1]);
         mbar_arrive(&s.qempty[q]);
       }
       advance(q, qph, nq);
@@ -1023,8 +1024,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     static_assert(kUnitInit + kUR < 64, "barrier initialisation needs more threads");
     const int i = threadIdx.x - 64;
     if (i >= 0 && i < kMaxNS) {
-      mbar_init(&s.full[i], 1);                // producer's arrive.expect_tx
-      mbar_init(&s.wfull[i], kDequantWarps);   // one arrival per dequant warp
+      // producer's arrive.expect_tx, then one arrival per dequant warp (INT8/INT4
+      // positions) or kDequantWarps more from the producer (BF16 positions)
+      mbar_init(&s.full[i], 1 + kDequantWarps);
       mbar_init(&s.empty[i], 1);               // tcgen05.commit
       mbar_init(&s.wfree[i], 1);               // producer, at INT8/INT4 positions
     } else if (i >= kMaxNS && i < kMaxNS + kMaxNQ) {
