@@ -201,7 +201,10 @@ def run_workload(cfg, steps, warmup, device, with_e2e, dist_barrier):
            "step_ms_all": t_step, "clocks": clk,
            "touched_bytes": float(np.mean([touched_bytes[i % n_batches] for i in range(steps)])),
            "io_bytes": io_bytes, "n_touched": float(np.mean(n_touched)),
-           "pairs": float(np.mean(pairs)), "launches_per_step": 6}
+           "pairs": float(np.mean(pairs)),
+           # this library's kernels per step: fused routing/grouping (T <= 128) or
+           # routing + grouping + gather, then the grouped FFN and the combine
+           "launches_per_step": 3 if cfg.T <= 128 else 5}
 
     if with_e2e:   # public API with host buffers: H2D inputs, forward, D2H output, every step
         pin = [(lg.pin_memory(), x.pin_memory()) for lg, x in host_batches]

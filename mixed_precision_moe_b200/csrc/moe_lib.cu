@@ -346,7 +346,43 @@ int set_ffn_attributes(int dev) {
   return MOE_OK;
 }
 
-// zero_counters = false: the caller has already zeroed the scheduler counters
+// Launch of route_permute_gather_kernel for moe_layer_forward (T <= 128).
+int route_permute_gather_small(moe_layer_t L, const float* logits, const void* x, int T,
+                               int renormalize, int32_t* topk_idx, float* topk_w,
+                               int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row,
+                               void* x_perm, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  const int E = L->E, k = L->k, H = L->H;
+  MOE_CHECK(logits && x && topk_idx && topk_w && expert_offsets && perm_token && dest_row &&
+                x_perm,
+            MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_CHECK(aligned(x, 16) && aligned(x_perm, 16), MOE_ERR_UNSUPPORTED,
+            "x and x_perm must be 16-byte aligned");
+  size_t need = 0;
+  moe_ffn_workspace_bytes(L, T * k, &need);
+  MOE_CHECK(workspace != nullptr && workspace_bytes >= need, MOE_ERR_INVALID_ARG,
+            "workspace %zu B < %zu B needed", workspace_bytes, need);
+  int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + need - kFfnCounterBytes);
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  const int pairs = T * k;
+  const int grid = std::max(1, std::min(2 * num_sms(dev), (pairs + 3) / 4));
+  const size_t smem = moe::front_smem_bytes(T, k, E);
+  const int keys = (E + 31) / 32;
+  auto kern = keys <= 1 ? moe::route_permute_gather_kernel<1>
+            : keys <= 2 ? moe::route_permute_gather_kernel<2>
+            : keys <= 4 ? moe::route_permute_gather_kernel<4>
+            : keys <= 8 ? moe::route_permute_gather_kernel<8>
+                        : moe::route_permute_gather_kernel<16>;
+  MOE_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(moe::kFrontThreads), smem, as_stream(stream),
+                          logits, static_cast<const uint4*>(x), T, E, k, renormalize, H / 8,
+                          topk_idx, topk_w, expert_offsets, perm_token, dest_row,
+                          static_cast<uint4*>(x_perm), counters,
+                          (int)(ffn_counter_bytes(E) / sizeof(int))));
+  return ok();
+}
+
+// zero_counters = false: the caller has already zeroed the scheduler counters// zero_counters = false: the caller has already zeroed the scheduler counters
 // on the stream (moe_layer_forward does so first, so that no memset node sits
 // between the layer's kernels).
 int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_offsets, int rows,
@@ -503,19 +539,29 @@ int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, 
                       int32_t* perm_token, int32_t* dest_row, void* x_perm, void* y_perm,
                       void* workspace, size_t workspace_bytes, void* out, void* stream) {
   MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
-  if (T > 0) {  // the FFN's scheduler counters, zeroed ahead of the layer's kernels
-    size_t need = 0;
-    moe_ffn_workspace_bytes(L, T * L->k, &need);
-    MOE_CHECK(workspace != nullptr && workspace_bytes >= need, MOE_ERR_INVALID_ARG,
-              "workspace %zu B < %zu B needed", workspace_bytes, need);
-    MOE_CUDA_TRY(cudaMemsetAsync(static_cast<uint8_t*>(workspace) + need - kFfnCounterBytes, 0,
-                                 ffn_counter_bytes(L->E), as_stream(stream)));
+  int rc = MOE_OK;
+  if (T > 0 && T <= moe::kFrontMaxTokens) {
+    // Small batch: routing, grouping and the row gather in one launch, which
+    // also zeroes the FFN's scheduler counters.
+    rc = route_permute_gather_small(L, logits, x, T, renormalize, topk_idx, topk_w,
+                                    expert_offsets, perm_token, dest_row, x_perm, workspace,
+                                    workspace_bytes, stream);
+    if (rc != MOE_OK) return rc;
+  } else {
+    if (T > 0) {  // the FFN's scheduler counters, zeroed ahead of the layer's kernels
+      size_t need = 0;
+      moe_ffn_workspace_bytes(L, T * L->k, &need);
+      MOE_CHECK(workspace != nullptr && workspace_bytes >= need, MOE_ERR_INVALID_ARG,
+                "workspace %zu B < %zu B needed", workspace_bytes, need);
+      MOE_CUDA_TRY(cudaMemsetAsync(static_cast<uint8_t*>(workspace) + need - kFfnCounterBytes, 0,
+                                   ffn_counter_bytes(L->E), as_stream(stream)));
+    }
+    rc = moe_route_topk(logits, T, L->E, L->k, renormalize, topk_idx, topk_w, stream);
+    if (rc != MOE_OK) return rc;
+    rc = moe_permute(topk_idx, x, T, L->E, L->k, L->H, expert_offsets, perm_token, dest_row,
+                     x_perm, stream);
+    if (rc != MOE_OK) return rc;
   }
-  int rc = moe_route_topk(logits, T, L->E, L->k, renormalize, topk_idx, topk_w, stream);
-  if (rc != MOE_OK) return rc;
-  rc = moe_permute(topk_idx, x, T, L->E, L->k, L->H, expert_offsets, perm_token, dest_row, x_perm,
-                   stream);
-  if (rc != MOE_OK) return rc;
   rc = grouped_ffn_impl(L, x_perm, expert_offsets, T * L->k, y_perm, workspace, workspace_bytes,
                         stream, false);
   if (rc != MOE_OK) return rc;

@@ -26,23 +26,16 @@ __device__ __forceinline__ float key_logit(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
-// One warp per token.  Lane l holds the keys of experts l, l+32, ... (KEYS
-// slots, ascending id).  k rounds of warp argmax pick the experts by
-// descending logit, ties to the lowest id; lane j keeps the j-th pick.
+// Top-k of one token by one warp.  Lane l holds the keys of experts l, l+32,
+// ... (KEYS slots, ascending id).  k rounds of warp argmax pick the experts by
+// descending logit, ties to the lowest id; lane j < k returns the j-th pick
+// and its gating weight.  nan_seen: some logit of the token was NaN (warp-wide).
 template <int KEYS>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
-                                                         int E, int k, int renormalize,
-                                                         int32_t* __restrict__ topk_idx,
-                                                         float* __restrict__ topk_w) {
-  pdl_launch_dependents();
-  pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  const float* z = logits + (size_t)t * E;
-
+__device__ __forceinline__ void route_token(const float* __restrict__ z, int E, int k,
+                                            int renormalize, int lane, int& pick_e,
+                                            float& pick_w, bool& nan_seen) {
   uint32_t key[KEYS];
-  bool nan_seen = false;
+  bool nan_here = false;
 #pragma unroll
   for (int i = 0; i < KEYS; ++i) {
     const int e = lane + 32 * i;
@@ -50,13 +43,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     if (e < E) {
       float v = z[e];
       if (isnan(v)) {
-        nan_seen = true;
+        nan_here = true;
         v = -INFINITY;
       }
       key[i] = logit_key(v);
     }
   }
-  if (__any_sync(0xffffffffu, nan_seen) && lane == 0) flag_status(MOE_STATUS_NONFINITE_LOGIT);
+  nan_seen = __any_sync(0xffffffffu, nan_here);
 
   int my_e = 0;
   float my_z = 0.0f;
@@ -100,9 +93,29 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     den = part;
   }
+  pick_e = my_e;
+  pick_w = ex / den;
+}
+
+// One warp per token.
+template <int KEYS>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
+                                                         int E, int k, int renormalize,
+                                                         int32_t* __restrict__ topk_idx,
+                                                         float* __restrict__ topk_w) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int e;
+  float w;
+  bool nan_seen;
+  route_token<KEYS>(logits + (size_t)t * E, E, k, renormalize, lane, e, w, nan_seen);
+  if (nan_seen && lane == 0) flag_status(MOE_STATUS_NONFINITE_LOGIT);
   if (lane < k) {
-    topk_idx[(size_t)t * k + lane] = my_e;
-    topk_w[(size_t)t * k + lane] = ex / den;
+    topk_idx[(size_t)t * k + lane] = e;
+    topk_w[(size_t)t * k + lane] = w;
   }
 }
 
@@ -257,6 +270,132 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
        i += (size_t)gridDim.x * blockDim.x) {
     const size_t r = i / vec_per_row, c = i % vec_per_row;
     x_perm[i] = x[(size_t)perm_token[r] * vec_per_row + c];
+  }
+}
+
+// ------------------------------------------- routing + grouping, small batch --
+
+constexpr int kFrontThreads = 1024;
+constexpr int kFrontMaxTokens = 128;
+
+__host__ __device__ constexpr size_t front_smem_bytes(int T, int k, int E) {
+  return (size_t)2 * T * k * sizeof(int32_t) + (size_t)2 * E * sizeof(int32_t);
+}
+
+// Routing, grouping and the row gather of a small batch (T <= 128) in one
+// launch, with the same results as route_topk_kernel + permute_index_kernel +
+// gather_rows_kernel.  Every CTA routes all T tokens into shared memory (a few
+// KB of logits) and derives the whole permutation, so no CTA waits for
+// another; CTA b then copies rows b, b + G, ... of x_perm, and CTA 0 alone
+// writes the index outputs and zeroes `zero_n` ints at `zero_ptr` (the FFN's
+// scheduler counters: after griddepcontrol.wait, so every earlier use of them
+// is complete).  Ids come from the routing above, so all are valid and
+// distinct within a token.
+template <int KEYS>
+__global__ void __launch_bounds__(kFrontThreads, 1)
+    route_permute_gather_kernel(const float* __restrict__ logits, const uint4* __restrict__ x,
+                                int T, int E, int k, int renormalize, int vec_per_row,
+                                int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+                                int32_t* __restrict__ dest_row, uint4* __restrict__ x_perm,
+                                int* __restrict__ zero_ptr, int zero_n) {
+  extern __shared__ int32_t fsm[];
+  const int pairs = T * k;
+  int32_t* sidx = fsm;                                     // [pairs] expert of pair (t, j)
+  int32_t* sperm = sidx + pairs;                           // [pairs] token of permuted row
+  int32_t* base = sperm + pairs;                           // [E]
+  uint32_t* mask = reinterpret_cast<uint32_t*>(base + E);  // [E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool lead = blockIdx.x == 0;
+  pdl_launch_dependents();
+  pdl_wait();
+
+  if (lead)
+    for (int i = tid; i < zero_n; i += blockDim.x) zero_ptr[i] = 0;
+  for (int i = tid; i < 2 * E; i += blockDim.x) base[i] = 0;  // base and mask
+
+  // 1. top-k: warp w routes tokens w, w + 32, ...
+  for (int t = warp; t < T; t += kFrontThreads / 32) {
+    int e;
+    float w;
+    bool nan_seen;
+    route_token<KEYS>(logits + (size_t)t * E, E, k, renormalize, lane, e, w, nan_seen);
+    if (lane < k) {
+      sidx[t * k + lane] = e;
+      if (lead) {
+        topk_idx[(size_t)t * k + lane] = e;
+        topk_w[(size_t)t * k + lane] = w;
+      }
+    }
+    if (lead && nan_seen && lane == 0) flag_status(MOE_STATUS_NONFINITE_LOGIT);
+  }
+  __syncthreads();
+
+  // 2. counts, exclusive scan, stable ranks (warp 0; order = expert id, then token)
+  if (warp == 0) {
+    for (int i = lane; i < pairs; i += 32) atomicAdd(&base[sidx[i]], 1);
+    __syncwarp();
+    const int per = (E + 31) / 32;
+    const int e0 = lane * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i)
+      if (e0 + i < E) local += base[e0 + i];
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    int run = incl - local;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < E) {
+        const int c = base[e];
+        base[e] = run;
+        if (lead) offsets[e] = run;
+        run += c;
+      }
+    }
+    if (lead && lane == 31) offsets[E] = incl;
+    __syncwarp();
+    const uint32_t lower = (1u << lane) - 1u;
+    for (int tb = 0; tb < T; tb += 32) {  // lane = token tb + lane
+      const int t = tb + lane;
+      const bool tv = t < T;
+      for (int j = 0; j < k; ++j)
+        if (tv) atomicOr(&mask[sidx[t * k + j]], 1u << lane);
+      __syncwarp();
+      for (int j = 0; j < k; ++j)
+        if (tv) {
+          const int e = sidx[t * k + j];
+          const int row = base[e] + __popc(mask[e] & lower);
+          sperm[row] = t;
+          if (lead) {
+            dest_row[(size_t)t * k + j] = row;
+            perm_token[row] = t;
+          }
+        }
+      __syncwarp();
+      for (int j = 0; j < k; ++j)
+        if (tv) {
+          const int e = sidx[t * k + j];
+          const uint32_t mm = mask[e];
+          if ((mm & lower) == 0) {  // lowest lane of this expert updates
+            base[e] += __popc(mm);
+            mask[e] = 0;
+          }
+        }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+
+  // 3. this CTA's rows of x_perm
+  const int G = gridDim.x;
+  const int rows_here = (pairs - (int)blockIdx.x + G - 1) / G;
+  for (int i = tid; i < rows_here * vec_per_row; i += blockDim.x) {
+    const int r = (int)blockIdx.x + (i / vec_per_row) * G, c = i % vec_per_row;
+    x_perm[(size_t)r * vec_per_row + c] = x[(size_t)sperm[r] * vec_per_row + c];
   }
 }
 
