@@ -18,7 +18,9 @@ same workload and value = all ranks' tokens / the slowest rank's time.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
+import re
 import os
 import subprocess
 import sys
@@ -40,6 +42,33 @@ def expert_bytes(prec, H, I):
     """Stored bytes of one expert (weights + fp16 group-128 scales)."""
     P = 3 * H * I
     return {synth.BF16: 2 * P, synth.INT8: P + P // 64, synth.INT4: P // 2 + P // 64}[int(prec)]
+
+
+FFN_SOURCES = ("grouped_ffn.cuh", "ptx.cuh", "common.cuh")
+FFN_PROFILE = os.path.join(ROOT, "profiles", "grouped_ffn_decode_qwen3_30b_b32.md")
+
+
+def ffn_kernel_hash():
+    h = hashlib.sha256()
+    for f in FFN_SOURCES:
+        with open(os.path.join(ROOT, "mixed_precision_moe_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ffn_traffic(bytes_per_launch):
+    """DRAM read + write bytes of one decode FFN launch from the committed ncu
+    capture, scaled to `bytes_per_launch` algorithmic bytes by the captured
+    launch's own algorithmic bytes; None if the kernel sources changed since."""
+    try:
+        text = open(FFN_PROFILE).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic-record: kernel_sha256=(\w+) dram_bytes=(\d+) algorithmic_bytes=(\d+)",
+                  text)
+    if not m or m.group(1) != ffn_kernel_hash():
+        return None
+    return int(m.group(2)) * bytes_per_launch / int(m.group(3))
 
 
 def load_peaks():
@@ -388,12 +417,14 @@ def main():
             "config": {"workload": workload_name(cfg), "global_batch": world * cfg.T,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between steps (256 MiB write)", "graph": "CUDA graph per step"},
-            "roofline": {"bound": "hbm", "kernel": "grouped FFN (gate/up + down launches)",
+            "roofline": {"bound": "hbm",
+                         "kernel": "grouped_ffn_kernel (gate/up + SwiGLU + down, one launch)",
                          "achieved": ffn_gbs, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": ffn_gbs / hbm_gbs, "frac_of_8000": ffn_gbs / 8000.0,
                          "bytes_per_launch": dec["touched_bytes"],
                          "touched_experts": dec["n_touched"],
-                         "peak_source": peak_src, "traffic": None},
+                         "peak_source": peak_src,
+                         "traffic": ffn_traffic(dec["touched_bytes"])},
             "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": dec["h2d_bytes"], "d2h_bytes_per_step": dec["d2h_bytes"]},
             "gpu_launches": dec["launches_per_step"] * args.steps,

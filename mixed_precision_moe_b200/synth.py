@@ -157,3 +157,8 @@ def stack_logits(layer: int, step: int) -> np.ndarray:
 
 def stack_x(layer: int, step: int) -> np.ndarray:
     return gen_x(STACK["T"], STACK["H"], STACK["seed"] * 100000 + 1000 * layer + step)
+
+
+def stack_master(layer: int, e: int):
+    """bf16 master weights of expert e of stack layer `layer`."""
+    return gen_expert_master(STACK["H"], STACK["I"], STACK["seed"] * 10 + layer, e)
