@@ -96,7 +96,7 @@ struct Params {
   const int32_t* offsets;  // [E+1]
   __nv_bfloat16* h;        // [rows][I]: gate/up output, down input
   __nv_bfloat16* y;        // [rows][H]: down output
-  int* counter;            // work counter, zero at launch
+  int* counter;            // work counter, zero at launch (unit = gridDim.x + count)
   int* done;               // [E] finished gate/up epilogue warps per expert, zero at launch
   int E, H, I;
   int nwb_gu, nwb_dn;      // weight blocks per expert of each projection
@@ -219,78 +219,77 @@ __device__ __forceinline__ int tiles_of(int n, const Params& p) {
   return n > 0 ? (n + p.xrows - 1) / p.xrows : 0;
 }
 
-// All threads stage (offset, rows, precision) of every expert in shared memory
-// (one round of global loads), then warp 0 lists the experts with rows, with
-// their first unit index, in descending time per unit: INT4 and INT8 units
-// (dequant- and latency-bound) before BF16 units, so the dynamic scheduler
-// approximates longest-processing-time-first and the tail is made of the
-// short units.  Unit indices: every gate/up unit in that order, then every
-// down unit in the same expert order.
+// The unit table, built by every CTA from expert_offsets and the precision
+// array: the experts with rows, with their first unit index, in descending time
+// per unit -- INT4, then INT8, then BF16 experts (dequant- and latency-bound
+// units before BF16 units), ascending id inside a class -- so the dynamic
+// scheduler approximates longest-processing-time-first and the tail is made of
+// the short units.  Unit indices: every gate/up unit in that order, then every
+// down unit in the same expert order.  Thread e handles expert e; a block-wide
+// scan (warp shuffles, then the warp totals) gives each expert its tile offset
+// and entry index within and across the classes.
 __device__ void build_entries(const Params& p, const Smem& s) {
-  int* t_off = reinterpret_cast<int*>(s.q_st);  // staging area is free until the mainloop
-  int* t_n = t_off + kMaxE;
-  int* t_prec = t_n + kMaxE;
-  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-    const int a = p.offsets[e], b = p.offsets[e + 1];
-    t_off[e] = a;
-    t_n[e] = b - a;
-    t_prec[e] = p.prec[e];
-  }
-  __syncthreads();
-  if ((threadIdx.x >> 5) != 0) return;
-  const int lane = threadIdx.x & 31;
-  const int per = (p.E + 31) / 32;
-  const int e0 = lane * per;
-  int tile_run = 0, ent_run = 0;
-  bool unset = false;
-  constexpr int kClassOrder[3] = {MOE_INT4, MOE_INT8, MOE_BF16};
-  for (int ci = 0; ci < 3; ++ci) {
-    const int cls = kClassOrder[ci];
-    int my_tiles = 0, my_ents = 0;
-    for (int i = 0; i < per; ++i) {
-      const int e = e0 + i;
-      if (e >= p.E) break;
-      const int n = t_n[e], prec = t_prec[e];
-      if (ci == 0 && n > 0 && (prec < MOE_BF16 || prec > MOE_INT4)) unset = true;
-      if (prec == cls && n > 0) {
-        my_tiles += tiles_of(n, p);
-        my_ents += 1;
-      }
+  static_assert(kThreads >= kMaxE, "one thread per expert");
+  constexpr int kWarps = kThreads / 32;
+  int* wsum = reinterpret_cast<int*>(s.q_st);  // [kWarps][6]; staging is free until the mainloop
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int off = 0, n = 0, prec = -1, cls = 3, tiles = 0;
+  if (tid < p.E) {
+    off = p.offsets[tid];
+    n = p.offsets[tid + 1] - off;
+    prec = p.prec[tid];
+    if (n > 0) {
+      cls = prec == MOE_INT4 ? 0 : prec == MOE_INT8 ? 1 : prec == MOE_BF16 ? 2 : 3;
+      if (cls == 3) flag_status(MOE_STATUS_UNSET_EXPERT);
+      tiles = tiles_of(n, p);
     }
-    int t_incl = my_tiles, e_incl = my_ents;
+  }
+  // v[c] = tiles of class c, v[3 + c] = entries of class c (this thread's expert)
+  int v[6];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    v[c] = cls == c ? tiles : 0;
+    v[3 + c] = cls == c ? 1 : 0;
+  }
+  int incl[6];
+#pragma unroll
+  for (int i = 0; i < 6; ++i) {
+    incl[i] = v[i];
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, t_incl, d);
-      const int b = __shfl_up_sync(0xffffffffu, e_incl, d);
-      if (lane >= d) {
-        t_incl += a;
-        e_incl += b;
-      }
+      const int x = __shfl_up_sync(0xffffffffu, incl[i], d);
+      if (lane >= d) incl[i] += x;
     }
-    int t = tile_run + t_incl - my_tiles, en = ent_run + e_incl - my_ents;
-    for (int i = 0; i < per; ++i) {
-      const int e = e0 + i;
-      if (e >= p.E) break;
-      const int n = t_n[e];
-      if (t_prec[e] == cls && n > 0) {
-        // tiles before this expert, times the weight blocks of each projection
-        s.entries[en] = Entry{t * p.nwb_gu, e | (cls << 16), t_off[e], n};
-        s.ub_dn[en] = t * p.nwb_dn;  // offset by the gate/up total below
-        t += tiles_of(n, p);
-        en += 1;
-      }
-    }
-    tile_run += __shfl_sync(0xffffffffu, t_incl, 31);
-    ent_run += __shfl_sync(0xffffffffu, e_incl, 31);
+    if (lane == 31) wsum[warp * 6 + i] = incl[i];
   }
-  const int total_gu = tile_run * p.nwb_gu;
-  __syncwarp();
-  for (int i = lane; i < ent_run; i += 32) s.ub_dn[i] += total_gu;
-  if (__any_sync(0xffffffffu, unset) && lane == 0) flag_status(MOE_STATUS_UNSET_EXPERT);
-  if (lane == 0) {
+  __syncthreads();
+  int before[6], total[6];  // sums over earlier warps / over all warps
+#pragma unroll
+  for (int i = 0; i < 6; ++i) before[i] = total[i] = 0;
+  for (int w = 0; w < kWarps; ++w)
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+      const int x = wsum[w * 6 + i];
+      total[i] += x;
+      if (w < warp) before[i] += x;
+    }
+  const int total_tiles = total[0] + total[1] + total[2];
+  const int total_gu = total_tiles * p.nwb_gu;
+  if (cls < 3) {
+    int tile_base = 0, ent_base = 0;
+    for (int c = 0; c < cls; ++c) {
+      tile_base += total[c];
+      ent_base += total[3 + c];
+    }
+    const int t = tile_base + before[cls] + incl[cls] - v[cls];
+    const int en = ent_base + before[3 + cls] + incl[3 + cls] - v[3 + cls];
+    s.entries[en] = Entry{t * p.nwb_gu, tid | (prec << 16), off, n};
+    s.ub_dn[en] = total_gu + t * p.nwb_dn;
+  }
+  if (tid == 0) {
     *s.n_units_gu = total_gu;
-    *s.n_units = total_gu + tile_run * p.nwb_dn;
-    *s.n_entries = ent_run;
+    *s.n_units = total_gu + total_tiles * p.nwb_dn;
+    *s.n_entries = total[3] + total[4] + total[5];
   }
 }
 
@@ -412,7 +411,8 @@ __device__ void scheduler(const Params& p, const Smem& s) {
       }
       gph ^= 1u;
     }
-    const int u = atomicAdd(p.counter, 1);
+    // the first unit of CTA b is unit b; later ones come from the counter
+    const int u = first ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.counter, 1);
     Unit un = Unit{0, 0, 0, 0, 0, 0, 0, 0};
     if (u < total) {
       un = decode_unit<kSwap>(p, s, u);
