@@ -17,6 +17,7 @@
 #include "route_permute_combine.cuh"
 
 namespace {
+constexpr int kMaxDevices = 64;  // per-device caches below
 
 thread_local std::string g_last_error;
 
@@ -283,19 +284,33 @@ int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int
   MOE_CHECK(aligned(x, 16) && aligned(x_perm, 16), MOE_ERR_UNSUPPORTED,
             "x and x_perm must be 16-byte aligned");
   const size_t smem = moe::permute_smem_bytes(E);
-  static bool attr_set = false;
-  if (!attr_set) {
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  static std::atomic<bool> attr_set[kMaxDevices];
+  if (dev >= kMaxDevices || !attr_set[dev].load()) {
     MOE_CUDA_TRY(cudaFuncSetAttribute(moe::permute_index_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)moe::permute_smem_bytes(512)));
-    attr_set = true;
+    if (dev < kMaxDevices) attr_set[dev].store(true);
   }
-  MOE_CUDA_TRY(launch_pdl(moe::permute_index_kernel, dim3(1), dim3(moe::kPermuteThreads), smem, s,
-                          topk_idx, T, E, k, expert_offsets, perm_token, dest_row));
+  if (T <= 2 * moe::kPermuteChunk) {  // one CTA
+    MOE_CUDA_TRY(launch_pdl(moe::permute_index_kernel, dim3(1), dim3(moe::kPermuteThreads), smem,
+                            s, topk_idx, T, E, k, expert_offsets, perm_token, dest_row,
+                            static_cast<const int32_t*>(nullptr)));
+  } else {
+    // Split over CTAs of kPermuteChunk tokens: per-CTA expert counts first.  They
+    // are kept in x_perm (nblk * E ints <= T * k * H * 2 bytes), which the row
+    // gather below overwrites only after the second pass has read them.
+    const int nblk = (T + moe::kPermuteChunk - 1) / moe::kPermuteChunk;
+    int32_t* counts = static_cast<int32_t*>(x_perm);
+    MOE_CUDA_TRY(launch_pdl(moe::permute_count_kernel, dim3(nblk), dim3(moe::kPermuteThreads),
+                            (size_t)E * sizeof(int32_t), s, topk_idx, T, E, k, counts));
+    MOE_CUDA_TRY(launch_pdl(moe::permute_index_kernel, dim3(nblk), dim3(moe::kPermuteThreads),
+                            smem, s, topk_idx, T, E, k, expert_offsets, perm_token, dest_row,
+                            static_cast<const int32_t*>(counts)));
+  }
   const int vec = H / 8;
   const long long nvec = (long long)T * k * vec;
-  int dev = 0;
-  MOE_CUDA_TRY(cudaGetDevice(&dev));
   const long long cap = (long long)num_sms(dev) * 8;
   const int blocks = (int)std::max(1LL, std::min(cap, (nvec + 255) / 256));
   MOE_CUDA_TRY(launch_pdl(moe::gather_rows_kernel, dim3(blocks), dim3(256), 0, s,
@@ -328,7 +343,6 @@ int moe_grouped_ffn_mixed(moe_layer_t L, const void* x_perm, const int32_t* expe
 }  // extern "C"
 
 namespace {
-constexpr int kMaxDevices = 64;
 
 // The kernel's dynamic shared-memory limit is a per-device function attribute;
 // it is set once per device.

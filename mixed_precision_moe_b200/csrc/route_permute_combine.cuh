@@ -124,35 +124,77 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 constexpr int kPermuteThreads = 1024;
 constexpr int kPermuteWarps = kPermuteThreads / 32;
 
+constexpr int kPermuteChunk = 256;   // tokens per CTA when the grouping is split over CTAs
+
 __host__ __device__ constexpr size_t permute_smem_bytes(int E) {
-  return (size_t)(2 * kPermuteWarps + 1) * E * sizeof(int32_t);
+  return (size_t)(2 * kPermuteWarps + 2) * E * sizeof(int32_t);
 }
 
-// Whole grouping in one CTA.  Warp w owns a contiguous chunk of tokens.
+// Large batches, first pass: CTA b counts the valid pairs of tokens
+// [b * kPermuteChunk, (b + 1) * kPermuteChunk) per expert into
+// blk_counts[b * E + e] (the same validity rule as permute_index_kernel).
+__global__ void __launch_bounds__(kPermuteThreads)
+    permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                         int32_t* __restrict__ blk_counts) {
+  extern __shared__ int32_t cnt[];
+  const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kPermuteChunk, t1 = min(T, t0 + kPermuteChunk);
+  for (int t = t0 + tid; t < t1; t += blockDim.x) {
+    int ev[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) ev[j] = (j < k) ? idx[(size_t)t * k + j] : -1;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j >= k) break;
+      bool ok = ev[j] >= 0 && ev[j] < E;
+#pragma unroll
+      for (int jj = 0; jj < j; ++jj) ok = ok && (ev[jj] != ev[j]);
+      if (ok) atomicAdd(&cnt[ev[j]], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) blk_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// Grouping of tokens [c0, c1) by one CTA; warp w owns a contiguous chunk.
 //   1. per-(warp, expert) counts (shared-memory atomics: order-free sums)
 //   2. exclusive scan over (expert, warp) -> expert_offsets and per-warp bases
 //   3. each warp walks its tokens 32 at a time in token order; a token's rank
 //      inside expert e is the number of lower lanes that also chose e, read
 //      from a per-(warp, expert) lane bitmask.
-// The resulting order (expert id, then token) is fixed; no atomic decides it.
+// One CTA (blk_counts == nullptr): c0 = 0, c1 = T.  Split over CTAs: CTA b
+// takes tokens [b * kPermuteChunk, ...) and adds, per expert, the pairs of all
+// experts below and of the CTAs before it (from permute_count_kernel), so the
+// result is the same.  The order (expert id, then token) is fixed; no atomic
+// decides it.
 __global__ void __launch_bounds__(kPermuteThreads, 1)
     permute_index_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
                          int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
-                         int32_t* __restrict__ dest_row) {
+                         int32_t* __restrict__ dest_row,
+                         const int32_t* __restrict__ blk_counts) {
   extern __shared__ int32_t psm[];
   int32_t* base = psm;                                          // [warps][E]
   uint32_t* mask = reinterpret_cast<uint32_t*>(psm + kPermuteWarps * E);  // [warps][E]
   int32_t* tot = psm + 2 * kPermuteWarps * E;                   // [E]
+  int32_t* pre = tot + E;                                       // [E] pairs of earlier CTAs
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool split = blk_counts != nullptr;
+  const bool lead = !split || blockIdx.x == 0;
   pdl_launch_dependents();
   pdl_wait();
 
   for (int i = tid; i < 2 * kPermuteWarps * E; i += blockDim.x) psm[i] = 0;
   __syncthreads();
 
-  const int chunk = (T + kPermuteWarps - 1) / kPermuteWarps;
-  const int t_begin = min(T, warp * chunk);
-  const int t_end = min(T, t_begin + chunk);
+  const int c0 = split ? (int)blockIdx.x * kPermuteChunk : 0;
+  const int c1 = split ? min(T, c0 + kPermuteChunk) : T;
+  const int chunk = (c1 - c0 + kPermuteWarps - 1) / kPermuteWarps;
+  const int t_begin = min(c1, c0 + warp * chunk);
+  const int t_end = min(c1, t_begin + chunk);
 
   // 1. counts of the valid pairs
   bool bad = false;
@@ -175,7 +217,8 @@ __global__ void __launch_bounds__(kPermuteThreads, 1)
   if (bad) flag_status(MOE_STATUS_BAD_EXPERT_ID);
   __syncthreads();
 
-  // 2a. per expert, exclusive prefix over warps
+  // 2a. per expert, exclusive prefix over warps; tot = this CTA's pairs, or
+  // with the split, all CTAs' pairs (pre = those of the CTAs before this one)
   for (int e = tid; e < E; e += blockDim.x) {
     int run = 0;
     for (int w = 0; w < kPermuteWarps; ++w) {
@@ -184,6 +227,16 @@ __global__ void __launch_bounds__(kPermuteThreads, 1)
       run += c;
     }
     tot[e] = run;
+    if (split) {
+      int all = 0, before = 0;
+      for (int b = 0; b < (int)gridDim.x; ++b) {
+        const int c = blk_counts[(size_t)b * E + e];
+        all += c;
+        if (b < (int)blockIdx.x) before += c;
+      }
+      tot[e] = all;
+      pre[e] = before;
+    }
   }
   __syncthreads();
   // 2b. exclusive scan of the expert totals (warp 0; lane owns a run of ids)
@@ -204,12 +257,12 @@ __global__ void __launch_bounds__(kPermuteThreads, 1)
       const int e = e0 + i;
       if (e < E) {
         const int c = tot[e];
-        tot[e] = run;
-        offsets[e] = run;
+        tot[e] = run + (split ? pre[e] : 0);
+        if (lead) offsets[e] = run;
         run += c;
       }
     }
-    if (lane == 31) offsets[E] = incl;
+    if (lead && lane == 31) offsets[E] = incl;
   }
   __syncthreads();
   for (int i = tid; i < kPermuteWarps * E; i += blockDim.x) base[i] += tot[i % E];

@@ -80,8 +80,10 @@ def test_route_nan_is_ordered_last_and_flagged():
 
 # -------------------------------------------------------------- permutation --
 
+# T > 512 takes the grouping split over CTAs of 256 tokens (ragged last chunk included)
 @pytest.mark.parametrize("T,E,k", [(64, 8, 2), (32, 128, 8), (4096, 128, 8), (32, 512, 10),
-                                   (1, 1, 1), (1000, 16, 16), (33, 300, 5)])
+                                   (1, 1, 1), (1000, 16, 16), (33, 300, 5), (2049, 300, 5),
+                                   (513, 512, 1)])
 def test_permute_bit_exact(T, E, k):
     H = 256
     logits = synth.gen_logits(T, E, 200 + T, 1.1)
@@ -99,8 +101,9 @@ def test_permute_bit_exact(T, E, k):
     assert _status() == 0
 
 
-def test_permute_invalid_and_repeated_ids():
-    T, E, k, H = 40, 6, 3, 128
+@pytest.mark.parametrize("T", [40, 1300])   # one CTA, split over CTAs
+def test_permute_invalid_and_repeated_ids(T):
+    E, k, H = 6, 3, 128
     rng = np.random.default_rng(3)
     idx = rng.integers(-2, E + 2, (T, k)).astype(np.int32)
     idx[5] = [1, 1, 2]
