@@ -313,6 +313,33 @@ def oracle_baseline(cfg, budget_s=10.0):
 
 # ----------------------------------------------------------------- main --
 
+def prefill_result(args, world, device, barrier, tf_burst, peak_src):
+    """The prefill workload (tile orientation, tensor-bound) as a JSON object."""
+    pcfg = synth.CONFIGS["qwen3_30b_prefill"]
+    pre = run_workload(pcfg, max(10, args.steps // 10), args.warmup, device, False, barrier)
+    p_step = max_over_ranks(pre["step_ms"], world, device)
+    p_ffn = max_over_ranks(pre["ffn_ms"], world, device)
+    flops = 6.0 * pcfg.H * pcfg.I * pre["pairs"]
+    tflops = flops / (p_ffn * 1e-3) / 1e12
+    return {"workload": workload_name(pcfg), "value": world * pcfg.T / (p_step * 1e-3),
+            "unit": "tokens/s", "ms_per_step": p_step, "ffn_ms": p_ffn,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_burst,
+                         "unit": "TFLOP/s", "frac": tflops / tf_burst,
+                         "frac_of_spec_2250": tflops / 2250.0,
+                         "flops_per_launch": flops, "peak_source": peak_src + " burst",
+                         "traffic": None},
+            "touched_experts": pre["n_touched"], "clocks": pre["clocks"]}
+
+
+def max_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -321,6 +348,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the prefill workload and print its object (for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -372,37 +401,22 @@ def main():
     barrier()
 
     hbm_gbs, tf_burst, tf_sust, peak_src = load_peaks()
+    if args.prefill_only:
+        pre = prefill_result(args, world, device, barrier, tf_burst, peak_src)
+        if rank == 0:
+            print(json.dumps(pre))
+        return
     dec = run_workload(cfg, args.steps, args.warmup, device, True, barrier)
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    step_ms = max_over_ranks(dec["step_ms"])
-    ffn_ms = max_over_ranks(dec["ffn_ms"])
-    e2e_ms = max_over_ranks(dec["e2e_ms"])
+    step_ms = max_over_ranks(dec["step_ms"], world, device)
+    ffn_ms = max_over_ranks(dec["ffn_ms"], world, device)
+    e2e_ms = max_over_ranks(dec["e2e_ms"], world, device)
     value = world * cfg.T / (step_ms * 1e-3)
     ffn_gbs = dec["touched_bytes"] / (ffn_ms * 1e-3) / 1e9
 
     prefill = None
     if not args.no_prefill:
-        pcfg = synth.CONFIGS["qwen3_30b_prefill"]
-        pre = run_workload(pcfg, max(10, args.steps // 10), args.warmup, device, False, barrier)
-        p_step = max_over_ranks(pre["step_ms"])
-        p_ffn = max_over_ranks(pre["ffn_ms"])
-        flops = 6.0 * pcfg.H * pcfg.I * pre["pairs"]
-        tflops = flops / (p_ffn * 1e-3) / 1e12
-        prefill = {"workload": workload_name(pcfg), "value": world * pcfg.T / (p_step * 1e-3),
-                   "unit": "tokens/s", "ms_per_step": p_step, "ffn_ms": p_ffn,
-                   "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_burst,
-                                "unit": "TFLOP/s", "frac": tflops / tf_burst,
-                                "frac_of_spec_2250": tflops / 2250.0,
-                                "flops_per_launch": flops, "peak_source": peak_src + " burst",
-                                "traffic": None},
-                   "touched_experts": pre["n_touched"], "clocks": pre["clocks"]}
+        prefill = prefill_result(args, world, device, barrier, tf_burst, peak_src)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
