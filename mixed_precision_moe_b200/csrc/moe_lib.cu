@@ -302,6 +302,8 @@ int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int
     // are kept in x_perm (nblk * E ints <= T * k * H * 2 bytes), which the row
     // gather below overwrites only after the second pass has read them.
     const int nblk = (T + moe::kPermuteChunk - 1) / moe::kPermuteChunk;
+    MOE_CHECK((size_t)T * k * H * 2 >= (size_t)nblk * E * sizeof(int32_t), MOE_ERR_UNSUPPORTED,
+              "x_perm too small to hold the grouping counts");
     int32_t* counts = static_cast<int32_t*>(x_perm);
     MOE_CUDA_TRY(launch_pdl(moe::permute_count_kernel, dim3(nblk), dim3(moe::kPermuteThreads),
                             (size_t)E * sizeof(int32_t), s, topk_idx, T, E, k, counts));
