@@ -130,7 +130,10 @@ int moe_route_topk(const float* logits, int T, int E, int k, int renormalize,
  *   perm_token     device int32 [T*k]: row -> token (rows >= offsets[E] unset)
  *   dest_row       device int32 [T][k]: pair -> row, or -1
  *   x_perm         device bf16 [T*k][H]: x_perm[r] = x[perm_token[r]]
- * Deterministic: no atomic decides any order. */
+ * Deterministic: no atomic decides any order.  For T > 512 the grouping is
+ * split over CTAs of 256 tokens (a count pass, then the ranking pass); the
+ * per-CTA counts are kept in x_perm until the row gather overwrites it, so
+ * x_perm is also written before the gather (it is an output either way). */
 int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int H,
                 int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row,
                 void* x_perm, void* stream);
@@ -198,7 +201,12 @@ int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w
  *   logits fp32 [T][E], x bf16 [T][H] -> out bf16 [T][H];
  *   scratch: topk_idx int32 [T][k], topk_w fp32 [T][k], expert_offsets int32
  *   [E+1], perm_token int32 [T*k], dest_row int32 [T][k], x_perm bf16
- *   [T*k][H], y_perm bf16 [T*k][H], workspace (moe_ffn_workspace_bytes). */
+ *   [T*k][H], y_perm bf16 [T*k][H], workspace (moe_ffn_workspace_bytes).
+ * For T <= 128 routing, grouping and the row gather run as one kernel (each
+ * CTA routes all T tokens in shared memory, then copies its share of x_perm
+ * rows); the outputs are identical to the separate calls.  The launches use
+ * programmatic dependent launch: each kernel may start while the previous one
+ * drains and waits (griddepcontrol.wait) before reading its inputs. */
 int moe_layer_forward(moe_layer_t layer, const float* logits, const void* x, int T,
                       int renormalize, int32_t* topk_idx, float* topk_w,
                       int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row,
