@@ -178,6 +178,25 @@ def time_graphs(graphs, steps, warmup, flush, stream):
     return [a.elapsed_time(b) for a, b in ev]
 
 
+def capture_layer_graphs(layer, dev_batches, bufs, stream):
+    """One graph per batch for the whole forward, and one for the grouped FFN alone."""
+    from mixed_precision_moe_b200 import binding as B
+    step_graphs, ffn_graphs = [], []
+    for b in range(len(dev_batches)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            layer.forward(*dev_batches[b], bufs=bufs[b], stream=stream)
+        step_graphs.append(g)
+        off, perm, dest, xp = bufs[b]["permute"]
+        y, ws = bufs[b]["ffn"]
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            B.moe_grouped_ffn_mixed(layer, xp, off, y, ws, stream=stream)
+        ffn_graphs.append(g2)
+    torch.cuda.synchronize()
+    return step_graphs, ffn_graphs
+
+
 def run_workload(cfg, steps, warmup, device, with_e2e, dist_barrier):
     """Returns a dict of timings and accounting for one layer config."""
     from mixed_precision_moe_b200 import binding as B
@@ -194,19 +213,7 @@ def run_workload(cfg, steps, warmup, device, with_e2e, dist_barrier):
             layer.forward(*dev_batches[b], bufs=bufs[b])
     torch.cuda.synchronize()
 
-    step_graphs, ffn_graphs = [], []
-    for b in range(n_batches):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            layer.forward(*dev_batches[b], bufs=bufs[b], stream=stream)
-        step_graphs.append(g)
-        off, perm, dest, xp = bufs[b]["permute"]
-        y, ws = bufs[b]["ffn"]
-        g2 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g2, stream=stream):
-            B.moe_grouped_ffn_mixed(layer, xp, off, y, ws, stream=stream)
-        ffn_graphs.append(g2)
-    torch.cuda.synchronize()
+    step_graphs, ffn_graphs = capture_layer_graphs(layer, dev_batches, bufs, stream)
 
     # algorithmic accounting from this run's routing (read back after the fact)
     touched_bytes, pairs, n_touched = [], [], []
@@ -327,6 +334,275 @@ def oracle_baseline(cfg, budget_s=10.0):
                       f"workload ({total:.1f} s), binary64 C oracle"}
 
 
+# ---------------------------------------------- secondary workloads --
+# Timing-only: their experts are drawn on the device (weights ~N(0, 0.02^2),
+# rounded to bf16) because the work does not depend on the values and the host
+# draw of several GB would dominate the run.  Parity on these shapes is covered
+# by the GPU tests with the host-drawn masters.
+
+def device_master(rows, K, gen, device, std=0.02):
+    return (torch.randn((rows, K), generator=gen, device=device) * std).to(torch.bfloat16)
+
+
+def mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src):
+    """Mixtral-8x7B-shaped layer, all experts INT4, uniform logits, over the
+    token batch sweep: per batch the layer step, the grouped FFN alone and the
+    FFN against its bound, max(expert bytes / HBM, flops / bf16 peak)."""
+    from mixed_precision_moe_b200 import binding as B
+    c0 = synth.mixtral_config(synth.MIXTRAL_BATCHES[0])
+    H, I, E, k = c0.H, c0.I, c0.E, c0.k
+    gen = torch.Generator(device=device)
+    gen.manual_seed(c0.seed)
+    layer = B.MoELayer(H, I, E, k)
+    for e in range(E):
+        w13 = device_master(2 * I, H, gen, device)
+        w2 = device_master(H, I, gen, device)
+        q13, s13 = B.moe_quantize_weights(w13, B.INT4)
+        q2, s2 = B.moe_quantize_weights(w2, B.INT4)
+        layer.set_expert(e, B.INT4, q13, s13, q2, s2)
+        del w13, w2
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    steps, warmup = max(10, args.steps // 4), args.warmup
+    eb = expert_bytes(synth.INT4, H, I)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    points = []
+    for T in synth.MIXTRAL_BATCHES:
+        cfg = synth.mixtral_config(T)
+        n_b = 2
+        dev_b = []
+        for b in range(n_b):
+            lg = synth.gen_logits(T, E, cfg.seed * 1000 + b)
+            x = synth.gen_x(T, H, cfg.seed * 1000 + b)
+            dev_b.append((torch.from_numpy(lg).to(device),
+                          torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)))
+        bufs = [layer.alloc_buffers(T, device) for _ in range(n_b)]
+        with torch.cuda.stream(stream):
+            for b in range(n_b):
+                layer.forward(*dev_b[b], bufs=bufs[b], stream=stream)
+        torch.cuda.synchronize()
+        step_g, ffn_g = capture_layer_graphs(layer, dev_b, bufs, stream)
+        t_step = time_graphs(step_g, steps, warmup, flush, stream)
+        t_ffn = time_graphs(ffn_g, steps, warmup, flush, stream)
+        d = [len(np.unique(bufs[b]["route"][0].cpu().numpy())) for b in range(n_b)]
+        d_mean = float(np.mean([d[i % n_b] for i in range(steps)]))
+        step_ms, ffn_ms = float(np.mean(t_step)), float(np.mean(t_ffn))
+        wbytes = d_mean * eb
+        flops = 6.0 * H * I * T * k
+        t_bytes = wbytes / (hbm_gbs * 1e9) * 1e3
+        t_flops = flops / (tf_burst * 1e12) * 1e3
+        if t_bytes >= t_flops:
+            bound, achieved, peak, unit = "hbm", wbytes / (ffn_ms * 1e-3) / 1e9, hbm_gbs, "GB/s"
+        else:
+            bound, achieved, peak, unit = ("tensor", flops / (ffn_ms * 1e-3) / 1e12, tf_burst,
+                                           "TFLOP/s")
+        points.append({"T": T, "tokens_per_s": T / (step_ms * 1e-3), "ms_per_step": step_ms,
+                       "ffn_ms": ffn_ms, "distinct_experts": d_mean, "expert_bytes": wbytes,
+                       "flops": flops, "bound": bound, "bound_ms": max(t_bytes, t_flops),
+                       "achieved": achieved, "peak": peak, "unit": unit,
+                       "frac": achieved / peak})
+        del step_g, ffn_g, bufs, dev_b
+    clk = clocks.stop()
+    status = B.moe_get_device_status()
+    if status:
+        raise RuntimeError(f"device status {status:#x} after the sweep")
+    layer.close()
+    return {"workload": f"mixtral_8x7b sweep: H={H} I={I} E={E} top-{k}, all experts INT4 "
+                        f"group-128, uniform N(0,1) logits, T in {list(synth.MIXTRAL_BATCHES)}",
+            "data": "synthetic (logits and x host-seeded; experts drawn on the device)",
+            "timing": f"CUDA graphs, {steps} timed replays after {warmup}, L2 flushed between",
+            "peaks": {"hbm_gbs": hbm_gbs, "bf16_tflops": tf_burst, "source": peak_src},
+            "points": points, "clocks": clk}
+
+
+def _hot_set(counts, n):
+    """The n most selected experts, ties to the lower id (sorted ids)."""
+    order = np.lexsort((np.arange(len(counts)), -counts))
+    return np.sort(order[:n])
+
+
+def stack_run(args, device, hbm_gbs, peak_src):
+    """Qwen3-80B-scale stack: 4 layers (H 2048, I 512, 512 experts, top-10) at
+    decode batch 32 for 256 steps, Zipf(1.2) routing whose popularity order is
+    redrawn every 64 steps.  Every expert stays resident as INT4; the 64
+    experts of each layer selected most often in the previous 64 steps are
+    BF16.  At each step 64 m the promoted experts' bf16 masters are copied from
+    pinned host memory on a side stream, the compute stream waits on that copy,
+    and every change goes through moe_set_expert_precision before the step's
+    forward.  A step is the four layer forwards (one CUDA graph each)."""
+    from mixed_precision_moe_b200 import binding as B
+    S = synth.STACK
+    nl, H, I, E, k, T = S["layers"], S["H"], S["I"], S["E"], S["k"], S["T"]
+    steps, epoch, n_hot = S["steps"], S["epoch"], S["n_hot"]
+    compute = torch.cuda.Stream(device)
+    copy = torch.cuda.Stream(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(S["seed"])
+    layers, int4, host13, host2, bf16, hot, prec_hist = [], [], [], [], [], [], []
+    chunk = 64
+    for l in range(nl):
+        L = B.MoELayer(H, I, E, k)
+        h13 = torch.empty((E, 2 * I, H), dtype=torch.bfloat16, pin_memory=True)
+        h2 = torch.empty((E, H, I), dtype=torch.bfloat16, pin_memory=True)
+        q = []
+        for e0 in range(0, E, chunk):
+            w13 = device_master(chunk * 2 * I, H, gen, device).view(chunk, 2 * I, H)
+            w2 = device_master(chunk * H, I, gen, device).view(chunk, H, I)
+            h13[e0:e0 + chunk].copy_(w13)
+            h2[e0:e0 + chunk].copy_(w2)
+            for j in range(chunk):
+                q.append(B.moe_quantize_weights(w13[j], B.INT4) +
+                         B.moe_quantize_weights(w2[j], B.INT4))
+            del w13, w2
+        first = set(np.argsort(synth.stack_ranks(l, 0), kind="stable")[:n_hot].tolist())
+        mine = {}
+        for e in range(E):
+            if e in first:
+                d13 = h13[e].to(device)
+                d2 = h2[e].to(device)
+                mine[e] = (d13, d2)
+                L.set_expert(e, B.BF16, d13, None, d2, None)
+            else:
+                q13, s13, q2, s2 = q[e]
+                L.set_expert(e, B.INT4, q13, s13, q2, s2)
+        layers.append(L)
+        int4.append(q)
+        host13.append(h13)
+        host2.append(h2)
+        bf16.append(mine)
+        hot.append(np.array(sorted(first)))
+    torch.cuda.synchronize()
+    prec_hist.append([np.isin(np.arange(E), hot[l]) for l in range(nl)])   # True = BF16
+
+    # every step's inputs on the device; routing of every step kept for the hot sets
+    lg_all = torch.empty((steps, nl, T, E), dtype=torch.float32, device=device)
+    x_all = torch.empty((steps, nl, T, H), dtype=torch.bfloat16, device=device)
+    for s in range(steps):
+        for l in range(nl):
+            lg_all[s, l].copy_(torch.from_numpy(synth.stack_logits(l, s)))
+            x_all[s, l].copy_(torch.from_numpy(synth.stack_x(l, s).view(np.int16))
+                              .view(torch.bfloat16))
+    hist = torch.zeros((steps, nl, T, k), dtype=torch.int32, device=device)
+    bufs = [layers[l].alloc_buffers(T, device) for l in range(nl)]
+    with torch.cuda.stream(compute):
+        for l in range(nl):
+            layers[l].forward(lg_all[0, l], x_all[0, l], bufs=bufs[l], stream=compute)
+    torch.cuda.synchronize()
+    pool = torch.cuda.graph_pool_handle()
+    graphs = []
+    with torch.cuda.stream(compute):
+        for s in range(steps):
+            row = []
+            for l in range(nl):
+                b = dict(bufs[l])
+                b["route"] = (hist[s, l], bufs[l]["route"][1])
+                g = torch.cuda.CUDAGraph()
+                g.capture_begin(pool=pool)
+                layers[l].forward(lg_all[s, l], x_all[s, l], bufs=b, stream=compute)
+                g.capture_end()
+                row.append(g)
+            graphs.append(row)
+    torch.cuda.synchronize()
+
+    def new_event():
+        return torch.cuda.Event(enable_timing=True)
+
+    with torch.cuda.stream(compute):
+        for i in range(args.warmup):
+            for g in graphs[0]:
+                g.replay()
+    torch.cuda.synchronize()
+    ev_s = [new_event() for _ in range(steps)]
+    ev_e = [new_event() for _ in range(steps)]
+    updates = []
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    with torch.cuda.stream(compute):
+        for s in range(steps):
+            if s > 0 and s % epoch == 0:
+                compute.synchronize()
+                sel = hist[s - epoch:s].cpu().numpy()
+                c0, c1 = new_event(), new_event()
+                plans, n_prom, n_dem = [], 0, 0
+                with torch.cuda.stream(copy):
+                    c0.record(copy)
+                    for l in range(nl):
+                        new_hot = _hot_set(np.bincount(sel[:, l].ravel(), minlength=E), n_hot)
+                        keep = set(new_hot.tolist())
+                        promote = [e for e in new_hot.tolist() if e not in bf16[l]]
+                        demote = [e for e in hot[l].tolist() if e not in keep]
+                        fresh = {e: (host13[l][e].to(device, non_blocking=True),
+                                     host2[l][e].to(device, non_blocking=True)) for e in promote}
+                        plans.append((l, promote, demote, fresh, new_hot))
+                        n_prom += len(promote)
+                        n_dem += len(demote)
+                    c1.record(copy)
+                compute.wait_event(c1)
+                for l, promote, demote, fresh, new_hot in plans:
+                    for e in demote:
+                        q13, s13, q2, s2 = int4[l][e]
+                        layers[l].set_expert(e, B.INT4, q13, s13, q2, s2, stream=compute)
+                        del bf16[l][e]
+                    for e in promote:
+                        bf16[l][e] = fresh[e]
+                        layers[l].set_expert(e, B.BF16, fresh[e][0], None, fresh[e][1], None,
+                                             stream=compute)
+                    hot[l] = new_hot
+                prec_hist.append([np.isin(np.arange(E), hot[l]) for l in range(nl)])
+                updates.append({"step": s, "promoted": n_prom, "demoted": n_dem,
+                                "h2d_bytes": n_prom * expert_bytes(synth.BF16, H, I),
+                                "copy": (c0, c1)})
+            ev_s[s].record(compute)
+            for g in graphs[s]:
+                g.replay()
+            ev_e[s].record(compute)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    status = B.moe_get_device_status()
+    if status:
+        raise RuntimeError(f"device status {status:#x} after the stack run")
+
+    step_ms = np.array([a.elapsed_time(b) for a, b in zip(ev_s, ev_e)])
+    total_ms = ev_s[0].elapsed_time(ev_e[-1])
+    upd_steps = {u["step"] for u in updates}
+    for u in updates:
+        u["gap_ms"] = ev_e[u["step"] - 1].elapsed_time(ev_s[u["step"]])
+        u["copy_ms"] = u["copy"][0].elapsed_time(u["copy"][1])
+        u["h2d_gbs"] = u["h2d_bytes"] / (u["copy_ms"] * 1e-3) / 1e9 if u["copy_ms"] > 0 else None
+        del u["copy"]
+    sel = hist.cpu().numpy()
+    touched = np.zeros(steps)
+    for s in range(steps):
+        bf = prec_hist[s // epoch]
+        for l in range(nl):
+            te = np.unique(sel[s, l])
+            nb = int(bf[l][te].sum())
+            touched[s] += nb * expert_bytes(synth.BF16, H, I) + \
+                (len(te) - nb) * expert_bytes(synth.INT4, H, I)
+    plain = np.array([s for s in range(steps) if s not in upd_steps])
+    mean_step = float(step_ms[plain].mean())
+    gbs = float(np.mean(touched[plain] / (step_ms[plain] * 1e-3) / 1e9))
+    del graphs
+    for L in layers:
+        L.close()
+    return {"workload": f"qwen3_80b_stack: {nl} layers x {steps} steps, H={H} I={I} E={E} "
+                        f"top-{k} T={T}, Zipf({S['zipf_s']}) popularity redrawn every {epoch} "
+                        f"steps, {n_hot} hottest BF16 per layer, every expert resident as INT4",
+            "data": "synthetic (logits and x host-seeded; experts drawn on the device)",
+            "timing": "CUDA events on the compute stream; a step is one CUDA graph per layer; "
+                      "no L2 flush (a step streams more than 1 GB of experts through the 126 MB L2)",
+            "tokens_per_s": T / (mean_step * 1e-3), "ms_per_step": mean_step,
+            "ms_per_layer": mean_step / nl,
+            "ms_per_step_p50": float(np.median(step_ms[plain])),
+            "ms_per_step_max": float(step_ms[plain].max()),
+            "tokens_per_s_with_updates": T * steps / (total_ms * 1e-3), "total_ms": total_ms,
+            "touched_bytes_per_step": float(touched[plain].mean()),
+            "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_gbs, "peak_source": peak_src,
+            "updates": updates, "clocks": clk}
+
+
 # ----------------------------------------------------------------- main --
 
 def prefill_result(args, world, device, barrier, tf_burst, peak_src):
@@ -366,6 +642,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill workload and print its object (for profiling)")
+    ap.add_argument("--workload", default="decode", choices=["decode", "mixtral-sweep", "stack"],
+                    help="decode: the headline line; mixtral-sweep / stack: one JSON object "
+                         "for that workload instead (one GPU)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -417,6 +696,14 @@ def main():
     barrier()
 
     hbm_gbs, tf_burst, tf_sust, peak_src = load_peaks()
+    if args.workload != "decode":
+        if world > 1:
+            raise SystemExit(f"--workload {args.workload} runs on one GPU")
+        if args.workload == "mixtral-sweep":
+            print(json.dumps(mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src)))
+        else:
+            print(json.dumps(stack_run(args, device, hbm_gbs, peak_src)))
+        return
     if args.prefill_only:
         pre = prefill_result(args, world, device, barrier, tf_burst, peak_src)
         if rank == 0:
