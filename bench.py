@@ -217,8 +217,10 @@ def run_workload(cfg, steps, warmup, device, with_e2e, dist_barrier):
 
     # algorithmic accounting from this run's routing (read back after the fact)
     touched_bytes, pairs, n_touched = [], [], []
+    selections = np.zeros(cfg.E, np.int64)
     for b in range(n_batches):
         idx = bufs[b]["route"][0].cpu().numpy()
+        selections += np.bincount(idx.ravel(), minlength=cfg.E)
         te = np.unique(idx)
         n_touched.append(len(te))
         touched_bytes.append(sum(expert_bytes(precs[e], cfg.H, cfg.I) for e in te))
@@ -237,7 +239,8 @@ def run_workload(cfg, steps, warmup, device, with_e2e, dist_barrier):
            "step_ms_all": t_step, "clocks": clk,
            "touched_bytes": float(np.mean([touched_bytes[i % n_batches] for i in range(steps)])),
            "io_bytes": io_bytes, "n_touched": float(np.mean(n_touched)),
-           "pairs": float(np.mean(pairs)),
+           "pairs": float(np.mean(pairs)), "n_batches": n_batches,
+           "selections": selections.tolist(),
            # this library's kernels per step: fused routing/grouping (T <= 128) or
            # routing + grouping + gather, then the grouped FFN and the combine
            "launches_per_step": 3 if cfg.T <= 128 else 5}
@@ -322,16 +325,27 @@ class OracleRunner:
         return len(tokens), time.perf_counter() - t0
 
 
-def oracle_baseline(cfg, budget_s=10.0):
-    """Time the CPU oracle on whole decode batches for about budget_s seconds."""
+def oracle_baseline(cfg, budget_s=10.0, single_s=3.0):
+    """Time the CPU oracle on whole decode batches for about budget_s seconds on
+    all host threads, then on 8-token slices for about single_s seconds on one."""
     r = OracleRunner(cfg)
     done, total = 0, 0.0
     while total < budget_s:
         n, dt = r.run(cfg.T)
         done, total = done + n, total + dt
+    one, t1, sl = 0, 0.0, 8
+    r.oracle.set_num_threads(1)
+    try:
+        while t1 < single_s:
+            n, dt = r.run(sl)
+            one, t1 = one + n, t1 + dt
+    finally:
+        r.oracle.set_num_threads(r.cores)
     return {"value": done / total, "unit": "tokens/s", "cores": r.cores, "kind": "oracle",
             "sample": f"{done // cfg.T} whole batches of {cfg.T} tokens of the {cfg.name} "
-                      f"workload ({total:.1f} s), binary64 C oracle"}
+                      f"workload ({total:.1f} s), binary64 C oracle",
+            "single_thread": {"value": one / t1, "unit": "tokens/s",
+                              "sample": f"{one // sl} slices of {sl} tokens ({t1:.1f} s)"}}
 
 
 # ---------------------------------------------- secondary workloads --
@@ -745,6 +759,8 @@ def main():
             "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": dec["h2d_bytes"], "d2h_bytes_per_step": dec["d2h_bytes"]},
             "gpu_launches": dec["launches_per_step"] * args.steps,
+            "routing": {"distinct_experts": dec["n_touched"], "batches": dec["n_batches"],
+                        "selections_per_expert": dec["selections"]},
             "clocks": dec["clocks"],
             "cpu_baseline": cpu,
             "prefill": prefill,

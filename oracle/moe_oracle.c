@@ -449,3 +449,13 @@ int oracle_num_threads(void) {
   return 1;
 #endif
 }
+
+/* Threads of the later parallel regions (n >= 1).  The work is split over
+ * (expert, row) and (token) only, so no result depends on it. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}

@@ -58,6 +58,11 @@ def num_threads() -> int:
     return int(_L().oracle_num_threads())
 
 
+def set_num_threads(n: int) -> None:
+    """OpenMP threads of later calls; results do not depend on the count."""
+    _L().oracle_set_num_threads(int(n))
+
+
 def bf16_to_double(b: int) -> float:
     return float(_L().oracle_bf16_to_double(int(b)))
 

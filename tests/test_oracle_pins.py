@@ -368,6 +368,26 @@ def test_layer_equals_route_permute_ffn_combine_and_numpy():
     assert np.allclose(out, ref, rtol=1e-11, atol=1e-14)
 
 
+def test_layer_result_does_not_depend_on_thread_count():
+    """The work is split over (expert, row) and tokens only: one thread and all
+    threads give the same bits (the timed CPU baseline reports both)."""
+    cfg = synth.CONFIGS["tiny"]
+    H, I, E, k, T = cfg.H, cfg.I, cfg.E, cfg.k, cfg.T
+    ex = _experts_from_master(H, I, E, cfg.seed, [oracle.INT4, oracle.INT8, oracle.BF16, oracle.INT4,
+                                                  oracle.INT8, oracle.BF16, oracle.INT4, oracle.INT4])
+    x = synth.gen_x(T, H, cfg.seed)
+    logits = synth.gen_logits(T, E, cfg.seed)
+    n = oracle.num_threads()
+    try:
+        oracle.set_num_threads(1)
+        one = oracle.moe_layer(logits, x, ex, k, H, I)
+    finally:
+        oracle.set_num_threads(n)
+    many = oracle.moe_layer(logits, x, ex, k, H, I)
+    for a, b in zip(one, many):
+        assert np.array_equal(a, b)
+
+
 # --------------------------------------------------------------- combine --
 
 def test_combine_one_hot_linearity_and_wave_split():
