@@ -40,6 +40,23 @@ MUTANTS = {
                           "load_row(ex->prec, ex->w2, ex->s2, I, I, m, row);"),
     "dropped_last_k_column": ("for (int c = 0; c < H; ++c) g += x[c] * row[c];",
                               "for (int c = 0; c < H - 1; ++c) g += x[c] * row[c];"),
+    "full_softmax_drops_first": ("for (int e = 0; e < E; ++e) den += exp((double)z[e] - m);",
+                                 "for (int e = 1; e < E; ++e) den += exp((double)z[e] - m);"),
+    "int8_q_128": ("const int Q = (prec == OR_INT4) ? 7 : 127;",
+                   "const int Q = (prec == OR_INT4) ? 7 : 128;"),
+    "fp16_subnormal_scale": ("v = ldexp((double)frac, -24);", "v = ldexp((double)frac, -25);"),
+    "up_reads_gate_rows": ("load_row(ex->prec, ex->w13, ex->s13, 2 * I, H, I + n, row);",
+                           "load_row(ex->prec, ex->w13, ex->s13, 2 * I, H, n, row);"),
+    "cursor_not_advanced": ("int row = cursor[e]++;", "int row = cursor[e];"),
+    "int4_offset_7": ("return u - 8;", "return u - 7;"),
+    "topk_ascending": ("if (best < 0 || z[e] > z[best]) best = e;",
+                       "if (best < 0 || z[e] < z[best]) best = e;"),
+    "duplicate_ids_kept": ("if (idx[(size_t)t * k + jj] == e) return 1;",
+                           "if (idx[(size_t)t * k + jj] == e + E) return 1;"),
+    "layer_weight_slot": ("double wj = w[(size_t)t * k + j];\n          for (int c = 0; c < H; ++c) o[c] += wj * y[c];",
+                          "double wj = w[(size_t)t * k + (j + 1) % k];\n          for (int c = 0; c < H; ++c) o[c] += wj * y[c];"),
+    "combine_weight_slot": ("double wj = w[(size_t)t * k + j];\n      for (int c = 0; c < H; ++c) o[c] += wj * y_perm",
+                            "double wj = w[(size_t)t * k + (j + 1) % k];\n      for (int c = 0; c < H; ++c) o[c] += wj * y_perm"),
 }
 
 
