@@ -726,6 +726,8 @@ def main():
     dec = run_workload(cfg, args.steps, args.warmup, device, True, barrier)
 
     step_ms = max_over_ranks(dec["step_ms"], world, device)
+    step_p50 = max_over_ranks(float(np.median(dec["step_ms_all"])), world, device)
+    step_p90 = max_over_ranks(float(np.percentile(dec["step_ms_all"], 90)), world, device)
     ffn_ms = max_over_ranks(dec["ffn_ms"], world, device)
     e2e_ms = max_over_ranks(dec["e2e_ms"], world, device)
     value = world * cfg.T / (step_ms * 1e-3)
@@ -743,6 +745,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "ms_per_step_p50": step_p50, "ms_per_step_p90": step_p90,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; Qwen3-30B-A3B-shaped layer, random-init experts)",
             "config": {"workload": workload_name(cfg), "global_batch": world * cfg.T,
