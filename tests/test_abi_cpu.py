@@ -81,3 +81,22 @@ def test_last_error_is_cleared_by_success(lib):
     assert _err(lib)
     assert lib.moe_combine(None, None, None, 0, 2, 256, None, None) == 0
     assert _err(lib) == ""
+
+
+def test_binding_refuses_host_tensors_instead_of_falling_back(lib):
+    """No CPU path exists: every entry point of the binding rejects tensors that
+    are not contiguous CUDA tensors of the expected dtype, before any library call."""
+    import torch
+    logits = torch.zeros((4, 8), dtype=torch.float32)
+    x = torch.zeros((4, 256), dtype=torch.bfloat16)
+    idx = torch.zeros((4, 2), dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.moe_route_topk(logits, 2)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.moe_permute(idx, x, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.moe_combine(x, idx, torch.zeros((4, 2)))
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.moe_quantize_weights(x, binding.INT4)
+    with pytest.raises(ValueError):
+        binding.moe_route_topk(logits.double(), 2)
