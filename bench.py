@@ -303,8 +303,6 @@ class OracleRunner:
 
     def __init__(self, cfg):
         import oracle
-        sys.path.insert(0, os.path.join(ROOT, "tests"))
-        from helpers import oracle_experts
         self.oracle, self.cfg = oracle, cfg
         ranks = synth.zipf_ranks(cfg.E, cfg.seed)
         precs = synth.precision_map(ranks, cfg.tiers)
@@ -313,7 +311,7 @@ class OracleRunner:
         idx = np.argsort(-self.logits, axis=1, kind="stable")[:, :cfg.k]
         needed = set(np.unique(idx).tolist())
         # unselected experts are never read; they stay in their bf16 master form
-        self.experts = oracle_experts(cfg.H, cfg.I, [precs[e] if e in needed else synth.BF16
+        self.experts = oracle.seeded_experts(cfg.H, cfg.I, [precs[e] if e in needed else synth.BF16
                                                      for e in range(cfg.E)], cfg.seed)
         self.cores = oracle.num_threads()
 

@@ -69,6 +69,7 @@ typedef enum { MOE_BF16 = 0, MOE_INT8 = 1, MOE_INT4 = 2 } moe_precision_t;
 #define MOE_STATUS_NONFINITE_LOGIT 0x2u /* a NaN logit (ordered as -inf) */
 #define MOE_STATUS_WAIT_TIMEOUT 0x4u   /* a kernel gave up a bounded wait */
 #define MOE_STATUS_UNSET_EXPERT 0x8u   /* FFN met an expert without weights */
+#define MOE_STATUS_BAD_ROW_INDEX 0x10u /* expert_offsets or dest_row outside [0, rows) */
 
 typedef struct moe_layer* moe_layer_t;
 
@@ -155,8 +156,10 @@ int moe_ffn_workspace_bytes(moe_layer_t layer, int rows, size_t* bytes);
  *   workspace      device, >= moe_ffn_workspace_bytes(rows) bytes, 256-byte
  *                  aligned; holds h and the tile scheduler's counters (zeroed
  *                  by the call itself).
- * Fails with MOE_ERR_NOT_MATERIALIZED if any expert was never set.  Calls that
- * share a workspace must not overlap on the device. */
+ * Fails with MOE_ERR_NOT_MATERIALIZED if any expert was never set.  An expert
+ * whose rows [offsets[e], offsets[e+1]) do not lie inside [0, rows) is left
+ * out (nothing of it is read or written) and flags MOE_STATUS_BAD_ROW_INDEX.
+ * Calls that share a workspace must not overlap on the device. */
 int moe_grouped_ffn_mixed(moe_layer_t layer, const void* x_perm,
                           const int32_t* expert_offsets, int rows, void* y_perm,
                           void* workspace, size_t workspace_bytes, void* stream);
@@ -174,7 +177,10 @@ int moe_grouped_ffn_mixed(moe_layer_t layer, const void* x_perm,
  *   rows * I * 2 + 4096 <= 8 MiB; larger calls fail with MOE_ERR_UNSUPPORTED.
  *   The first call on a device looks up the scratch's device address (a
  *   cudaGetSymbolAddress with that device current); make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is cached per device index for
+ *   the life of the process: after cudaDeviceReset (or with another context
+ *   made current on that device) call moe_ffn_noalloc_reset() before the next
+ *   call, so the address is looked up again.
  *   All calls on a device share the one scratch array, which keeps the last
  *   call's contents (the call zeroes the counters it needs): calls that
  *   overlap on the GPU (different streams, or several layers in flight) race
@@ -186,11 +192,17 @@ int moe_grouped_ffn_mixed_noalloc(moe_layer_t layer, const void* x_perm,
 /* Size in bytes of the scratch array behind moe_grouped_ffn_mixed_noalloc. */
 int moe_ffn_noalloc_max_bytes(size_t* bytes);
 
+/* Forget the cached scratch address of the current device (see above); the
+ * next moe_grouped_ffn_mixed_noalloc call on it looks the address up again. */
+int moe_ffn_noalloc_reset(void);
+
 /* Weighted combine back to token order (ExactMoE Section 3.4; weights are not
  * renormalised): out[t] = sum_j topk_w[t][j] * y_perm[dest_row[t][j]] in fp32,
  * j in order 0..k-1, pairs with dest_row < 0 skipped, one rounding to bf16.
- *   y_perm device bf16 [rows][H]; dest_row device int32 [T][k];
- *   topk_w device fp32 [T][k]; out device bf16 [T][H]. */
+ *   y_perm device bf16 [rows][H] with rows = T*k; dest_row device int32
+ *   [T][k]; topk_w device fp32 [T][k]; out device bf16 [T][H].
+ * A dest_row >= T*k is skipped and flags MOE_STATUS_BAD_ROW_INDEX (no read
+ * outside y_perm). */
 int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w,
                 int T, int k, int H, void* out, void* stream);
 

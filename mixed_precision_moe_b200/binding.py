@@ -17,6 +17,7 @@ STATUS_BAD_EXPERT_ID = 0x1
 STATUS_NONFINITE_LOGIT = 0x2
 STATUS_WAIT_TIMEOUT = 0x4
 STATUS_UNSET_EXPERT = 0x8
+STATUS_BAD_ROW_INDEX = 0x10
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
@@ -35,6 +36,7 @@ SIGNATURES = {
     "moe_grouped_ffn_mixed": (_I, [_P, _P, _P, _I, _P, _P, _S, _P]),
     "moe_grouped_ffn_mixed_noalloc": (_I, [_P, _P, _P, _I, _P, _P]),
     "moe_ffn_noalloc_max_bytes": (_I, [C.POINTER(_S)]),
+    "moe_ffn_noalloc_reset": (_I, []),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_layer_forward": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _P]),
     "moe_quantize_weights": (_I, [_P, _I, _I, _I, _P, _P, _P]),
@@ -56,13 +58,15 @@ _lib = None
 
 
 def lib():
-    """Load libmoe.so (built in-tree by mixed_precision_moe_b200.build)."""
+    """Load libmoe.so (built in-tree by mixed_precision_moe_b200.build), or the
+    library named by MOE_LIB_PATH (the profiling build of ffn_trace.py)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"libmoe.so is not built ({LIB_PATH}); run "
+        path = os.environ.get("MOE_LIB_PATH") or LIB_PATH
+        if not os.path.exists(path):
+            raise RuntimeError(f"libmoe.so is not built ({path}); run "
                                "`python -m mixed_precision_moe_b200.build`")
-        L = C.CDLL(LIB_PATH)
+        L = C.CDLL(path)
         for name, (res, args) in SIGNATURES.items():
             f = getattr(L, name)
             f.restype, f.argtypes = res, args
@@ -161,6 +165,12 @@ def moe_ffn_noalloc_max_bytes() -> int:
     n = C.c_size_t(0)
     _check(lib().moe_ffn_noalloc_max_bytes(C.byref(n)))
     return n.value
+
+
+def moe_ffn_noalloc_reset():
+    """Forget the cached scratch address of the current device (after a device
+    reset); the next no-alloc call looks it up again."""
+    _check(lib().moe_ffn_noalloc_reset())
 
 
 def moe_combine(y_perm, dest_row, topk_w, out=None, stream=None):

@@ -98,6 +98,7 @@ struct Params {
   __nv_bfloat16* y;        // [rows][H]: down output
   int* counter;            // work counter, zero at launch (unit = gridDim.x + count)
   int* done;               // [E] finished gate/up epilogue warps per expert, zero at launch
+  int rows;                // row capacity of x_perm, h and y_perm
   int E, H, I;
   int nwb_gu, nwb_dn;      // weight blocks per expert of each projection
   int xbox_rows;           // rows per X tensor-map box
@@ -114,6 +115,51 @@ struct SmemMap {
 };
 
 constexpr int kNumBarriers = 96;
+
+// ------------------------------------------------------------------- trace --
+// Profiling builds only (-DMOE_FFN_TRACE): a per-CTA, per-unit record written
+// by every role -- absolute stamps (%globaltimer, ns) and the SM cycles a role
+// spent waiting on its barriers for the unit (clock64 sums).  Unit `seq` is the
+// CTA's seq-th valid unit; every role receives the units in the same order.
+// Read back with moe_ffn_trace_read; the normal build compiles all of it away.
+enum TraceField {
+  kTrUnit = 0,     // global unit index
+  kTrKind,         // flags | prec << 8 | nrows << 16 | expert << 24
+  kTrSched,        // ns: scheduler published the unit
+  kTrProdBeg,      // ns: producer took the unit
+  kTrProdEnd,      // ns: producer issued the unit's last copies
+  kTrProdWait,     // cycles: producer waiting on empty
+  kTrCodeWait,     // cycles: code producer waiting on qempty
+  kTrMmaBeg,       // ns: MMA thread, accumulator buffer free
+  kTrMmaEnd,       // ns: MMA thread, last commit issued
+  kTrMmaWait,      // cycles: MMA thread waiting on full
+  kTrDqBeg,        // ns: dequant warp 2, unit taken (INT8/INT4)
+  kTrDqEnd,        // ns: dequant warp 2, last slot handed over
+  kTrDqWaitQ,      // cycles: dequant warp 2 waiting on qfull
+  kTrDqWaitW,      // cycles: dequant warp 2 waiting on wfree
+  kTrEpiBeg,       // ns: epilogue warp 4, accumulator full
+  kTrEpiEnd,       // ns: epilogue warp 4, rows stored
+  kTraceFields
+};
+#ifdef MOE_FFN_TRACE
+constexpr int kTraceCtas = 160, kTraceUnits = 96;
+__device__ long long g_ffn_trace[kTraceCtas][kTraceUnits][kTraceFields];
+__device__ __forceinline__ void trace_set(int seq, int f, long long v) {
+  if (blockIdx.x < kTraceCtas && seq < kTraceUnits) g_ffn_trace[blockIdx.x][seq][f] = v;
+}
+__device__ __forceinline__ void trace_add(int seq, int f, long long v) {
+  if (blockIdx.x < kTraceCtas && seq < kTraceUnits) g_ffn_trace[blockIdx.x][seq][f] += v;
+}
+#define FFN_TRACE_SET(seq, f, v) trace_set((seq), (f), (long long)(v))
+#define FFN_TRACE_ADD(seq, f, v) trace_add((seq), (f), (long long)(v))
+#define FFN_TRACE_NS() ((long long)global_timer_ns())
+#define FFN_CLOCK() clock64()
+#else
+#define FFN_TRACE_SET(seq, f, v) ((void)0)
+#define FFN_TRACE_ADD(seq, f, v) ((void)0)
+#define FFN_TRACE_NS() 0ll
+#define FFN_CLOCK() 0ll
+#endif
 
 __host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows, int E) {
   SmemMap m;
@@ -245,6 +291,12 @@ __device__ void build_entries(const Params& p, const Smem& s) {
     off = p.offsets[tid];
     n = p.offsets[tid + 1] - off;
     prec = p.prec[tid];
+    // An expert whose rows do not lie inside [0, rows) is left out (no unit
+    // reads or writes them) and flagged: the epilogue's stores use these rows.
+    if (off < 0 || n < 0 || off > p.rows || n > p.rows - off) {
+      if (n != 0) flag_status(MOE_STATUS_BAD_ROW_INDEX);
+      n = 0;
+    }
     if (n > 0) {
       if (prec == MOE_INT4 || prec == MOE_INT8 || prec == MOE_BF16) {
         cls = kSwap ? 0 : (prec == MOE_INT4 ? 0 : prec == MOE_INT8 ? 1 : 2);
@@ -419,6 +471,8 @@ __device__ void scheduler(const Params& p, const Smem& s) {
   volatile int* abort_flag = s.abort_flag;
   const int total = *s.n_units;
   uint32_t us = 0, uph = 0, gph = 0;
+  int tseq = 0;
+  (void)tseq;
   bool ok = true;
   for (bool first = true;; first = false) {
     if (!first) {
@@ -448,6 +502,11 @@ __device__ void scheduler(const Params& p, const Smem& s) {
     mbar_arrive(&s.ufull[us]);
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
+    FFN_TRACE_SET(tseq, kTrUnit, u);
+    FFN_TRACE_SET(tseq, kTrKind,
+                  un.flags | un.prec << 8 | un.nrows << 16 | (long long)un.e << 24);
+    FFN_TRACE_SET(tseq, kTrSched, FFN_TRACE_NS());
+    ++tseq;
   }
   if (!ok) give_up(s);
 }
@@ -464,6 +523,8 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
   uint32_t issued = 0, issued_par = 0;  // drain bookkeeping
   const uint32_t xbytes = (uint32_t)p.xbox_rows * 128;
   bool ok = true;
+  int tseq = 0;
+  (void)tseq;
   prefetch_tmap(tm_x);
   prefetch_tmap(tm_h);
   for (;;) {
@@ -475,6 +536,7 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
     mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
+    FFN_TRACE_SET(tseq, kTrProdBeg, FFN_TRACE_NS());
 
     const bool gu = unit_gu(un);
     const ExpertDesc* d = p.descs + un.e;
@@ -488,10 +550,12 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
     const int reserve_kb = max(0, nkb - (int)ns - 4);
     for (int kb = 0; kb < nkb; ++kb) {
       if (kb == reserve_kb) mbar_arrive(s.go);
+      const long long c0 = FFN_CLOCK();
       if (!mbar_wait(&s.empty[st], sph ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
+      FFN_TRACE_ADD(tseq, kTrProdWait, FFN_CLOCK() - c0);
       if (!bf16) mbar_arrive(&s.wfree[st]);  // the dequant warps may fill this stage
       mbar_arrive_expect_tx(&s.full[st], bytes);
       if (bf16) mbar_arrive_n(&s.full[st], kDequantWarps);  // no dequant at this position
@@ -505,6 +569,8 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
       advance(st, sph, ns);
     }
     if (!ok) break;
+    FFN_TRACE_SET(tseq, kTrProdEnd, FFN_TRACE_NS());
+    ++tseq;
   }
   if (!ok) {
     give_up(s);
@@ -527,6 +593,8 @@ __device__ void code_producer(const Params& p, const Smem& s) {
   uint32_t q = 0, qph = 0, us = 0, uph = 0;
   uint32_t qissued = 0, qissued_par = 0;  // drain bookkeeping
   bool ok = true;
+  int tseq = -1;
+  (void)tseq;
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
       ok = false;
@@ -536,6 +604,7 @@ __device__ void code_producer(const Params& p, const Smem& s) {
     mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
+    ++tseq;
     if (un.prec == MOE_BF16) continue;
     const bool gu = unit_gu(un);
     const ExpertDesc* d = p.descs + un.e;
@@ -545,10 +614,12 @@ __device__ void code_producer(const Params& p, const Smem& s) {
     const int nkb = unit_nkb(p, un);
     const bool int4 = un.prec == MOE_INT4;
     for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
+      const long long c0 = FFN_CLOCK();
       if (!mbar_wait(&s.qempty[q], qph ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
+      FFN_TRACE_ADD(tseq, kTrCodeWait, FFN_CLOCK() - c0);
       mbar_arrive_expect_tx(&s.qfull[q], (uint32_t)un.nbox * (kBoxRows * 64 + kBoxRows * 2));
       const int kc = int4 ? (kb >> 1) * 64 : kb * 64;  // byte column of the codes
       const int g = kb >> 1;                            // K-group of the scales
@@ -608,6 +679,8 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
   uint32_t st = 0, sph = 0, us = 0, uph = 0, abuf = 0;
   uint32_t aph[2] = {0, 0};
   bool ok = true;
+  int tseq = 0;
+  (void)tseq;
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
       ok = false;
@@ -623,16 +696,19 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
       break;
     }
     tc_fence_after();
+    FFN_TRACE_SET(tseq, kTrMmaBeg, FFN_TRACE_NS());
     const uint32_t d_tmem = tmem + abuf * acc_cols;
     const int n = kSwap ? max(16, (un.nrows + 15) & ~15) : un.nbox * kBoxRows;
     const uint32_t idesc = idesc_bf16_f32(128, n);
     const bool quant = un.prec != MOE_BF16;
     const bool a_in_tmem = kSwap && quant;  // dequantised weights live in TMEM
     for (int kb = 0; kb < nkb; ++kb) {
+      const long long c0 = FFN_CLOCK();
       if (!mbar_wait(&s.full[st], sph, abort_flag)) {  // X landed, weights in place
         ok = false;
         break;
       }
+      FFN_TRACE_ADD(tseq, kTrMmaWait, FFN_CLOCK() - c0);
       tc_fence_after();
       const uint64_t xd = xdesc0 + st * xstep, wd = wdesc0 + st * wstep;
       const uint32_t acc0 = kb != 0;
@@ -647,6 +723,8 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
     }
     if (!ok) break;
     mma_commit(&s.accfull[abuf]);
+    FFN_TRACE_SET(tseq, kTrMmaEnd, FFN_TRACE_NS());
+    ++tseq;
     aph[abuf] ^= 1u;
     abuf ^= 1u;
   }
@@ -727,6 +805,10 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
   uint32_t fph = 0;  // wfree phase bit per stage: it only advances on INT8/INT4 positions
   bool ok = true;
+  int tseq = -1;
+  const bool tracer = warp == 2 && lane == 0;
+  (void)tseq;
+  (void)tracer;
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
       ok = false;
@@ -737,11 +819,13 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
     if (lane == 0) mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
+    ++tseq;
     const int nkb = unit_nkb(p, un);
     if (un.prec == MOE_BF16) {
       for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
       continue;
     }
+    if (tracer) FFN_TRACE_SET(tseq, kTrDqBeg, FFN_TRACE_NS());
     const bool int4 = un.prec == MOE_INT4;
     const float off = int4 ? 32776.0f : 32896.0f;  // 2^15 + 8, 2^15 + 128
     for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
@@ -749,11 +833,20 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
       advance(st, sph, ns);
       const uint32_t st1 = st;
       if (int4) advance(st, sph, ns);
-      if (!mbar_wait(&s.qfull[q], qph, abort_flag) ||
-          !mbar_wait(&s.wfree[st0], (fph >> st0) & 1u, abort_flag) ||
+      const long long tq0 = FFN_CLOCK();
+      if (!mbar_wait(&s.qfull[q], qph, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const long long tq1 = FFN_CLOCK();
+      if (!mbar_wait(&s.wfree[st0], (fph >> st0) & 1u, abort_flag) ||
           (int4 && !mbar_wait(&s.wfree[st1], (fph >> st1) & 1u, abort_flag))) {
         ok = false;
         break;
+      }
+      if (tracer) {
+        FFN_TRACE_ADD(tseq, kTrDqWaitQ, tq1 - tq0);
+        FFN_TRACE_ADD(tseq, kTrDqWaitW, FFN_CLOCK() - tq1);
       }
       fph ^= (1u << st0) | (int4 ? 1u << st1 : 0u);
       tc_fence_after();
@@ -792,6 +885,7 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
       advance(q, qph, nq);
     }
     if (!ok) break;
+    if (tracer) FFN_TRACE_SET(tseq, kTrDqEnd, FFN_TRACE_NS());
   }
   if (!ok) give_up(s);
 }
@@ -920,6 +1014,10 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
   uint32_t us = 0, uph = 0, ebuf = 0, xph = 0;
   uint32_t eph[2] = {0, 0};
   bool ok = true;
+  int tseq = 0;
+  const bool tracer = warp == 4 && lane == 0;
+  (void)tseq;
+  (void)tracer;
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
       ok = false;
@@ -936,6 +1034,7 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
       break;
     }
     tc_fence_after();
+    if (tracer) FFN_TRACE_SET(tseq, kTrEpiBeg, FFN_TRACE_NS());
     const uint32_t tb = tmem + ((uint32_t)(quarter * 32) << 16) + ebuf * acc_cols;
     if (kSwap) {
       const int wr = quarter * 32 + lane;  // weight row of the unit (TMEM lane)
@@ -1021,6 +1120,8 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.accempty[ebuf]);
     if (gu) publish_rows(p, un, lane);
+    if (tracer) FFN_TRACE_SET(tseq, kTrEpiEnd, FFN_TRACE_NS());
+    ++tseq;
     eph[ebuf] ^= 1u;
     ebuf ^= 1u;
   }

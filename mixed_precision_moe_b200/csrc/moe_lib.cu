@@ -173,6 +173,25 @@ const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 int moe_abi_version(void) { return 1; }
 
+#ifdef MOE_FFN_TRACE
+// Profiling builds only (not part of moe.h): the grouped FFN's per-unit record.
+size_t moe_ffn_trace_bytes(void) { return sizeof(moe::ffn::g_ffn_trace); }
+
+int moe_ffn_trace_reset(void) {
+  void* addr = nullptr;
+  MOE_CUDA_TRY(cudaGetSymbolAddress(&addr, moe::ffn::g_ffn_trace));
+  MOE_CUDA_TRY(cudaMemset(addr, 0, sizeof(moe::ffn::g_ffn_trace)));
+  return ok();
+}
+
+int moe_ffn_trace_read(void* host_dst, size_t bytes) {
+  MOE_CHECK(host_dst != nullptr && bytes <= sizeof(moe::ffn::g_ffn_trace), MOE_ERR_INVALID_ARG,
+            "bad trace buffer");
+  MOE_CUDA_TRY(cudaMemcpyFromSymbol(host_dst, moe::ffn::g_ffn_trace, bytes));
+  return ok();
+}
+#endif
+
 int moe_layer_create(int H, int I, int E, int k, moe_layer_t* out) {
   MOE_CHECK(out != nullptr, MOE_ERR_INVALID_ARG, "out is null");
   *out = nullptr;
@@ -362,6 +381,26 @@ int set_ffn_attributes(int dev) {
   return MOE_OK;
 }
 
+// Every host-side check of the grouped FFN, so that moe_layer_forward can run
+// them before it enqueues anything.
+int ffn_check(moe_layer_t L, const void* x_perm, const int32_t* expert_offsets, int rows,
+              const void* y_perm, const void* workspace, size_t workspace_bytes) {
+  MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  MOE_CHECK(rows >= 0, MOE_ERR_INVALID_ARG, "rows=%d < 0", rows);
+  if (rows == 0) return MOE_OK;
+  MOE_CHECK(x_perm && expert_offsets && y_perm && workspace, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_CHECK(aligned(x_perm, 16) && aligned(y_perm, 16), MOE_ERR_UNSUPPORTED,
+            "x_perm and y_perm must be 16-byte aligned");
+  MOE_CHECK(aligned(workspace, 256), MOE_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+  size_t need = 0;
+  moe_ffn_workspace_bytes(L, rows, &need);
+  MOE_CHECK(workspace_bytes >= need, MOE_ERR_INVALID_ARG, "workspace %zu B < %zu B needed",
+            workspace_bytes, need);
+  for (int e = 0; e < L->E; ++e)
+    MOE_CHECK(L->prec[e] >= 0, MOE_ERR_NOT_MATERIALIZED, "expert %d has no weights", e);
+  return MOE_OK;
+}
+
 // Launch of route_permute_gather_kernel for moe_layer_forward (T <= 128).
 int route_permute_gather_small(moe_layer_t L, const float* logits, const void* x, int T,
                                int renormalize, int32_t* topk_idx, float* topk_w,
@@ -398,26 +437,17 @@ int route_permute_gather_small(moe_layer_t L, const float* logits, const void* x
   return ok();
 }
 
-// zero_counters = false: the caller has already zeroed the scheduler counters// zero_counters = false: the caller has already zeroed the scheduler counters
+// zero_counters = false: the caller has already zeroed the scheduler counters
 // on the stream (moe_layer_forward does so first, so that no memset node sits
 // between the layer's kernels).
 int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_offsets, int rows,
                      void* y_perm, void* workspace, size_t workspace_bytes, void* stream,
                      bool zero_counters) {
   using namespace moe::ffn;
-  MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
-  MOE_CHECK(rows >= 0, MOE_ERR_INVALID_ARG, "rows=%d < 0", rows);
-  if (rows == 0) return ok();
-  MOE_CHECK(x_perm && expert_offsets && y_perm && workspace, MOE_ERR_INVALID_ARG, "null pointer");
-  MOE_CHECK(aligned(x_perm, 16) && aligned(y_perm, 16), MOE_ERR_UNSUPPORTED,
-            "x_perm and y_perm must be 16-byte aligned");
-  MOE_CHECK(aligned(workspace, 256), MOE_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+  int rc = ffn_check(L, x_perm, expert_offsets, rows, y_perm, workspace, workspace_bytes);
+  if (rc != MOE_OK || rows == 0) return rc;
   size_t need = 0;
   moe_ffn_workspace_bytes(L, rows, &need);
-  MOE_CHECK(workspace_bytes >= need, MOE_ERR_INVALID_ARG, "workspace %zu B < %zu B needed",
-            workspace_bytes, need);
-  for (int e = 0; e < L->E; ++e)
-    MOE_CHECK(L->prec[e] >= 0, MOE_ERR_NOT_MATERIALIZED, "expert %d has no weights", e);
 
   cudaStream_t s = as_stream(stream);
   int dev = 0;
@@ -452,7 +482,7 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
   MOE_CHECK(smem <= kSmemLimit, MOE_ERR_UNSUPPORTED, "shared memory plan does not fit");
 
   CUtensorMap tm_x, tm_h;
-  int rc = encode_2d(&tm_x, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->H, xbox, 64,
+  rc = encode_2d(&tm_x, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->H, xbox, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != MOE_OK) return rc;
   rc = encode_2d(&tm_h, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->I, xbox, 64,
@@ -460,7 +490,7 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
   if (rc != MOE_OK) return rc;
 
   Params prm{L->d_descs, L->d_prec, expert_offsets, h, static_cast<__nv_bfloat16*>(y_perm),
-             counters, counters + 16, L->E, L->H, L->I,
+             counters, counters + 16, rows, L->E, L->H, L->I,
              swap ? L->I / 64 : L->I / 128, swap ? L->H / 128 : (L->H + 255) / 256,
              xbox, xrows, ns, nq, acc_stride, a_col};
 
@@ -532,6 +562,15 @@ int moe_ffn_noalloc_max_bytes(size_t* bytes) {
   return ok();
 }
 
+int moe_ffn_noalloc_reset(void) {
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  MOE_CHECK(dev >= 0 && dev < kMaxDevices, MOE_ERR_UNSUPPORTED, "device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  g_scratch_addr[dev] = nullptr;
+  return ok();
+}
+
 int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w, int T, int k,
                 int H, void* out, void* stream) {
   MOE_CHECK(T >= 0, MOE_ERR_INVALID_ARG, "T=%d < 0", T);
@@ -545,7 +584,7 @@ int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w
   const dim3 block(std::min(256, ((vec + 31) / 32) * 32));
   const dim3 grid(T, (vec + block.x - 1) / block.x);
   MOE_CUDA_TRY(launch_pdl(moe::combine_kernel, grid, block, 0, as_stream(stream),
-                          static_cast<const uint4*>(y_perm), dest_row, topk_w, k, vec,
+                          static_cast<const uint4*>(y_perm), dest_row, topk_w, k, vec, T * k,
                           static_cast<uint4*>(out)));
   return ok();
 }
@@ -555,8 +594,22 @@ int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, 
                       int32_t* perm_token, int32_t* dest_row, void* x_perm, void* y_perm,
                       void* workspace, size_t workspace_bytes, void* out, void* stream) {
   MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
-  int rc = MOE_OK;
-  if (T > 0 && T <= moe::kFrontMaxTokens) {
+  MOE_CHECK(T >= 0, MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0) {  // as the separate calls: no rows, every expert empty
+    MOE_CHECK(expert_offsets != nullptr, MOE_ERR_INVALID_ARG, "null expert_offsets");
+    MOE_CUDA_TRY(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (L->E + 1),
+                                 as_stream(stream)));
+    return ok();
+  }
+  // Every check of every step first, so that a call that fails has enqueued
+  // nothing and written no output.
+  int rc = ffn_check(L, x_perm, expert_offsets, T * L->k, y_perm, workspace, workspace_bytes);
+  if (rc != MOE_OK) return rc;
+  MOE_CHECK(logits && x && topk_idx && topk_w && perm_token && dest_row && out,
+            MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_CHECK(aligned(x, 16) && aligned(out, 16), MOE_ERR_UNSUPPORTED,
+            "x and out must be 16-byte aligned");
+  if (T <= moe::kFrontMaxTokens) {
     // Small batch: routing, grouping and the row gather in one launch, which
     // also zeroes the FFN's scheduler counters.
     rc = route_permute_gather_small(L, logits, x, T, renormalize, topk_idx, topk_w,
@@ -564,14 +617,11 @@ int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, 
                                     workspace_bytes, stream);
     if (rc != MOE_OK) return rc;
   } else {
-    if (T > 0) {  // the FFN's scheduler counters, zeroed ahead of the layer's kernels
-      size_t need = 0;
-      moe_ffn_workspace_bytes(L, T * L->k, &need);
-      MOE_CHECK(workspace != nullptr && workspace_bytes >= need, MOE_ERR_INVALID_ARG,
-                "workspace %zu B < %zu B needed", workspace_bytes, need);
-      MOE_CUDA_TRY(cudaMemsetAsync(static_cast<uint8_t*>(workspace) + need - kFfnCounterBytes, 0,
-                                   ffn_counter_bytes(L->E), as_stream(stream)));
-    }
+    // the FFN's scheduler counters, zeroed ahead of the layer's kernels
+    size_t need = 0;
+    moe_ffn_workspace_bytes(L, T * L->k, &need);
+    MOE_CUDA_TRY(cudaMemsetAsync(static_cast<uint8_t*>(workspace) + need - kFfnCounterBytes, 0,
+                                 ffn_counter_bytes(L->E), as_stream(stream)));
     rc = moe_route_topk(logits, T, L->E, L->k, renormalize, topk_idx, topk_w, stream);
     if (rc != MOE_OK) return rc;
     rc = moe_permute(topk_idx, x, T, L->E, L->k, L->H, expert_offsets, perm_token, dest_row,

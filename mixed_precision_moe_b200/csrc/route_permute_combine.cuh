@@ -418,25 +418,32 @@ __global__ void __launch_bounds__(kFrontThreads, 1)
       for (int j = 0; j < k; ++j)
         if (tv) atomicOr(&mask[sidx[t * k + j]], 1u << lane);
       __syncwarp();
-      for (int j = 0; j < k; ++j)
-        if (tv) {
-          const int e = sidx[t * k + j];
-          const int row = base[e] + __popc(mask[e] & lower);
+      // Every lane reads the masks of all its experts before any lane updates
+      // base/mask (the __syncwarp between the two loops), so the update never
+      // depends on how the lanes' j iterations interleave.
+      int ev[16];
+      uint32_t mm[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        ev[j] = -1;
+        mm[j] = 0;
+        if (tv && j < k) {
+          ev[j] = sidx[t * k + j];
+          mm[j] = mask[ev[j]];
+          const int row = base[ev[j]] + __popc(mm[j] & lower);
           sperm[row] = t;
           if (lead) {
             dest_row[(size_t)t * k + j] = row;
             perm_token[row] = t;
           }
         }
+      }
       __syncwarp();
-      for (int j = 0; j < k; ++j)
-        if (tv) {
-          const int e = sidx[t * k + j];
-          const uint32_t mm = mask[e];
-          if ((mm & lower) == 0) {  // lowest lane of this expert updates
-            base[e] += __popc(mm);
-            mask[e] = 0;
-          }
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (ev[j] >= 0 && (mm[j] & lower) == 0) {  // lowest lane of this expert updates
+          base[ev[j]] += __popc(mm[j]);
+          mask[ev[j]] = 0;
         }
       __syncwarp();
     }
@@ -465,10 +472,13 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 
 // out[t] = sum_j w[t][j] * y[dest_row[t][j]] in fp32, j = 0..k-1 in order.
 // grid (T, ceil(H/8 / blockDim.x)); each thread one 16-byte vector of a row.
+// Pairs with dest_row < 0 are skipped; a row >= rows (the capacity of y,
+// T * k) is skipped too and flagged, so no read leaves y.
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y,
                                                       const int32_t* __restrict__ dest_row,
                                                       const float* __restrict__ topk_w, int k,
-                                                      int vec_per_row, uint4* __restrict__ out) {
+                                                      int vec_per_row, int rows,
+                                                      uint4* __restrict__ out) {
   pdl_launch_dependents();
   pdl_wait();
   const int t = blockIdx.x;
@@ -478,6 +488,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   for (int j = 0; j < k; ++j) {
     const int r = dest_row[(size_t)t * k + j];
     if (r < 0) continue;
+    if (r >= rows) {
+      if (c == 0) flag_status(MOE_STATUS_BAD_ROW_INDEX);
+      continue;
+    }
     const float wj = topk_w[(size_t)t * k + j];
     float f[8];
     bf16x8_to_f32(y[(size_t)r * vec_per_row + c], f);

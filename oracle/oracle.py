@@ -191,3 +191,22 @@ def moe_layer(logits: np.ndarray, x: np.ndarray, experts, k: int, H: int, I: int
                                  w13, s13, w2, s2, tp, n, _p(idx), _p(w), _p(out)), "moe_layer")
     del keep
     return idx, w, out
+
+
+def seeded_experts(H: int, I: int, precs, seed: int, masters=None):
+    """The oracle-side experts of a seeded workload: each expert's bf16 master
+    (from the shared seeded input generators, or `masters[e]` if given) kept as
+    is for BF16, or quantised by this oracle's own group-128 quantiser for
+    INT8/INT4.  The GPU side receives exactly these codes and scales."""
+    from mixed_precision_moe_b200 import synth   # seeded generators only, no method arithmetic
+    out = []
+    for e, p in enumerate(precs):
+        w13, w2 = masters[e] if masters is not None else synth.gen_expert_master(H, I, seed, e)
+        p = int(p)
+        if p == BF16:
+            out.append(Expert(p, w13, None, w2, None))
+        else:
+            q13, s13 = quantize(w13, p)
+            q2, s2 = quantize(w2, p)
+            out.append(Expert(p, q13, s13, q2, s2))
+    return out

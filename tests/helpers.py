@@ -16,17 +16,7 @@ MAX_ABS_TOL = 1e-2      # max|gpu - oracle| <= MAX_ABS_TOL * max|oracle|
 
 
 def oracle_experts(H, I, precs, seed, masters=None):
-    out = []
-    for e, p in enumerate(precs):
-        w13, w2 = masters[e] if masters is not None else synth.gen_expert_master(H, I, seed, e)
-        p = int(p)
-        if p == oracle.BF16:
-            out.append(oracle.Expert(p, w13, None, w2, None))
-        else:
-            q13, s13 = oracle.quantize(w13, p)
-            q2, s2 = oracle.quantize(w2, p)
-            out.append(oracle.Expert(p, q13, s13, q2, s2))
-    return out
+    return oracle.seeded_experts(H, I, precs, seed, masters)
 
 
 def to_gpu_bf16(bits):
