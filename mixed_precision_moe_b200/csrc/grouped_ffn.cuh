@@ -46,6 +46,15 @@
 //     weight row.  The tensor core does no work on padding rows and the small
 //     X tiles leave room for a deep weight pipeline, so decode streams weight
 //     bytes; the gate/up epilogue exchanges the up half through shared memory.
+// CUDA-core units (swap mode): an INT8/INT4 expert with at most fma_rows rows
+// (the cold experts of a decode batch, one to a few tokens each) is not run on
+// the tensor core, whose rate at such small N is set by the A operand (128 x
+// 16 weights per MMA) and falls below the HBM rate of 4-bit weights.  Its units
+// flow through the same operand ring -- the producer stages 16 KB of codes, the
+// unit's X rows and the group scales per stage, so the ring keeps its full
+// depth of bytes in flight -- and the dequant warps compute exact fp32 dot
+// products from the codes (f32x2 FMAs); the MMA thread, the epilogue and the
+// code producer pass over them.
 #pragma once
 
 #include "common.cuh"
@@ -65,15 +74,28 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 232448; // dynamic shared memory per block on sm_100
 constexpr long long kDrainCycles = 2000000;  // ~1 ms: bound of a wait in the give-up path
 
+// CUDA-core units: token tiles of at most kFmaRows rows; one stage holds 128
+// weight rows x 128 code bytes (INT4: 256 K-elements, INT8: 128), then in the
+// X part the tile's X rows (kFmaRows x 128 bf16 per 128 K) and the group scales.
+constexpr int kFmaRows = 2;
+constexpr int kFmaXBytes = 2 * kFmaRows * 256;     // X of an INT4 stage (two 128-K boxes)
+constexpr int kFmaScaleBytes = 2 * kBoxRows * 2;   // fp16 scales of two K-groups
+constexpr int kFmaXStageMin =                      // X part of a stage, 1024-aligned
+    (kFmaXBytes + kFmaScaleBytes + 1023) / 1024 * 1024;
+
 struct alignas(64) ExpertDesc {
-  CUtensorMap tm_w13;  // codes/values of [2I][H] as [2][I][H]; box 2 x 64 rows x (64 bf16 | 64 B)
-  CUtensorMap tm_w2;   // codes/values of [H][I]; box 128 rows x (64 bf16 | 64 B)
-  const __half* s13;   // [H/128][2I]
-  const __half* s2;    // [I/128][H]
-  int prec;            // MOE_BF16 / MOE_INT8 / MOE_INT4, -1 when unset
+  CUtensorMap tm_w13;   // codes/values of [2I][H] as [2][I][H]; box 2 x 64 rows x (64 bf16 | 64 B)
+  CUtensorMap tm_w2;    // codes/values of [H][I]; box 128 rows x (64 bf16 | 64 B)
+  CUtensorMap tm_q13f;  // INT8/INT4 codes of W13 as [2][I][K bytes]; box 2 x 64 rows x 128 B
+  CUtensorMap tm_q2f;   // INT8/INT4 codes of W2; box 128 rows x 128 B
+  CUtensorMap tm_s13f;  // INT8/INT4 scales [H/128][2I] as [G][2][I]; box (INT4: 2, INT8: 1) x 2 x 64
+  CUtensorMap tm_s2f;   // INT8/INT4 scales [I/128][H]; box (2 | 1) groups x 128 rows
+  const __half* s13;    // [H/128][2I]
+  const __half* s2;     // [I/128][H]
+  int prec;             // MOE_BF16 / MOE_INT8 / MOE_INT4, -1 when unset
   int pad[11];
 };
-static_assert(sizeof(ExpertDesc) == 320, "descriptor layout");
+static_assert(sizeof(ExpertDesc) == 832, "descriptor layout");
 
 struct Unit {
   int e, prec, wrow0, nbox;  // expert, precision, first weight row (of each half), 128-row boxes
@@ -81,7 +103,7 @@ struct Unit {
   int flags;                 // kUnitValid | kUnitGateUp
   int need;                  // down unit: gate/up epilogue arrivals to wait for
 };
-constexpr int kUnitValid = 1, kUnitGateUp = 2;
+constexpr int kUnitValid = 1, kUnitGateUp = 2, kUnitFma = 4;
 
 struct Entry {
   int unit_begin;  // first gate/up unit index of this expert
@@ -106,6 +128,7 @@ struct Params {
   int ns, nq;              // ring depths
   int acc_stride;          // TMEM columns per accumulator buffer
   int a_col;               // swap mode: TMEM column of the first A stage (32 columns each)
+  int fma_rows;            // swap mode: INT8/INT4 experts with <= fma_rows rows run on CUDA cores
 };
 
 // Shared-memory map (byte offsets from the 1024-aligned base).
@@ -115,6 +138,9 @@ struct SmemMap {
 };
 
 constexpr int kNumBarriers = 96;
+// full, empty, wfree, fdone, ffull per stage; qfull, qempty per slot; accfull,
+// accempty; ufull, uempty; mmadone, xfull, xempty, go
+static_assert(5 * kMaxNS + 2 * kMaxNQ + 2 * 2 + 2 * kUR + 4 <= kNumBarriers, "barrier space");
 
 // ------------------------------------------------------------------- trace --
 // Profiling builds only (-DMOE_FFN_TRACE): a per-CTA, per-unit record written
@@ -139,6 +165,10 @@ enum TraceField {
   kTrDqWaitW,      // cycles: dequant warp 2 waiting on wfree
   kTrEpiBeg,       // ns: epilogue warp 4, accumulator full
   kTrEpiEnd,       // ns: epilogue warp 4, rows stored
+  kTrMmaIssue,     // cycles: MMA thread issuing (fence, MMAs, commit)
+  kTrDqConv,       // cycles: dequant warp 2 loading and converting codes
+  kTrDqStore,      // cycles: dequant warp 2 storing to TMEM and signalling (CUDA-core: output)
+  kTrPublish,      // cycles: the gate/up publication (fences + release add)
   kTraceFields
 };
 #ifdef MOE_FFN_TRACE
@@ -147,25 +177,23 @@ __device__ long long g_ffn_trace[kTraceCtas][kTraceUnits][kTraceFields];
 __device__ __forceinline__ void trace_set(int seq, int f, long long v) {
   if (blockIdx.x < kTraceCtas && seq < kTraceUnits) g_ffn_trace[blockIdx.x][seq][f] = v;
 }
-__device__ __forceinline__ void trace_add(int seq, int f, long long v) {
-  if (blockIdx.x < kTraceCtas && seq < kTraceUnits) g_ffn_trace[blockIdx.x][seq][f] += v;
-}
 #define FFN_TRACE_SET(seq, f, v) trace_set((seq), (f), (long long)(v))
-#define FFN_TRACE_ADD(seq, f, v) trace_add((seq), (f), (long long)(v))
 #define FFN_TRACE_NS() ((long long)global_timer_ns())
 #define FFN_CLOCK() clock64()
 #else
 #define FFN_TRACE_SET(seq, f, v) ((void)0)
-#define FFN_TRACE_ADD(seq, f, v) ((void)0)
 #define FFN_TRACE_NS() 0ll
 #define FFN_CLOCK() 0ll
 #endif
+// Cycle sums are kept in registers during a unit and stored once at its end
+// (a global read-modify-write per stage would itself stall the role).
 
 __host__ __device__ inline SmemMap smem_map(bool swap, int ns, int nq, int xrows, int E) {
   SmemMap m;
   const uint32_t wrows = swap ? 128 : 256;
   m.wstage = wrows * 128;
   m.xstage = (uint32_t)xrows * 128;
+  if (swap && m.xstage < (uint32_t)kFmaXStageMin) m.xstage = kFmaXStageMin;  // CUDA-core X + scales
   m.qslot = wrows * 64;
   m.qscale = wrows * 2;
   uint32_t off = 0;
@@ -196,7 +224,7 @@ struct Smem {
   uint8_t *w_st, *x_st, *q_st, *q_sc;
   float* xbuf;
   uint64_t *full, *empty, *wfree, *qfull, *qempty, *accfull, *accempty, *ufull, *uempty;
-  uint64_t *mmadone, *xfull, *xempty, *go;
+  uint64_t *mmadone, *xfull, *xempty, *go, *fdone, *ffull;
   Unit* units;
   uint32_t* tmem_slot;
   int* abort_flag;
@@ -232,6 +260,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const Params& p, bool swap) 
   s.xfull = s.mmadone + 1;
   s.xempty = s.xfull + 1;
   s.go = s.xempty + 1;
+  s.fdone = s.go + 1;
+  s.ffull = s.fdone + kMaxNS;
   s.units = reinterpret_cast<Unit*>(b + m.units);
   s.tmem_slot = reinterpret_cast<uint32_t*>(b + m.misc);
   s.abort_flag = reinterpret_cast<int*>(b + m.misc + 4);
@@ -254,7 +284,37 @@ __device__ __forceinline__ void advance(uint32_t& slot, uint32_t& phase, uint32_
   }
 }
 
-__device__ __forceinline__ void give_up(const Smem& s) {
+#ifdef MOE_FFN_TRACE
+// Profiling builds: per CTA, %globaltimer at kernel entry, after the barrier
+// and TMEM set-up, after the unit table, at the final barrier and at exit.
+__device__ long long g_ffn_kstamp[kTraceCtas][5];
+#define FFN_KSTAMP(i)                                                          \
+  do {                                                                        \
+    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas)                          \
+      g_ffn_kstamp[blockIdx.x][i] = (long long)global_timer_ns();              \
+  } while (0)
+#else
+#define FFN_KSTAMP(i) ((void)0)
+#endif
+
+#ifdef MOE_FFN_TRACE
+// Profiling builds: the role and unit of the first give-up of each CTA
+// ({role, unit sequence number, unit index of that role's last unit}).
+__device__ int g_ffn_giveup[kTraceCtas][4];
+#endif
+
+// role: 1 scheduler, 2 producer, 3 code producer, 4 MMA, 5 dequant, 6 epilogue
+__device__ __forceinline__ void give_up(const Smem& s, int role = 0, int seq = -1) {
+#ifdef MOE_FFN_TRACE
+  if (blockIdx.x < kTraceCtas && *reinterpret_cast<volatile int*>(s.abort_flag) == 0 &&
+      atomicCAS(&g_ffn_giveup[blockIdx.x][0], 0, role) == 0) {
+    g_ffn_giveup[blockIdx.x][1] = seq;
+    g_ffn_giveup[blockIdx.x][2] = threadIdx.x;
+  }
+#else
+  (void)role;
+  (void)seq;
+#endif
   *reinterpret_cast<volatile int*>(s.abort_flag) = 1;
   flag_status(MOE_STATUS_WAIT_TIMEOUT);
 }
@@ -279,8 +339,11 @@ __device__ __forceinline__ int tiles_of(int n, const Params& p) {
 //     3 % faster there than id order).
 // Thread e handles expert e; a block-wide scan (warp shuffles, then the warp
 // totals) gives each expert its tile offset and entry index.
+// my_prec: p.prec[threadIdx.x] (read by the caller before griddepcontrol.wait:
+// the precisions are written only by write_desc_kernel, which never lets a
+// dependent launch start before it completes).
 template <bool kSwap>
-__device__ void build_entries(const Params& p, const Smem& s) {
+__device__ void build_entries(const Params& p, const Smem& s, int my_prec) {
   static_assert(kThreads >= kMaxE, "one thread per expert");
   constexpr int kWarps = kThreads / 32;
   constexpr int kC = kSwap ? 1 : 3;            // classes in unit order
@@ -290,7 +353,7 @@ __device__ void build_entries(const Params& p, const Smem& s) {
   if (tid < p.E) {
     off = p.offsets[tid];
     n = p.offsets[tid + 1] - off;
-    prec = p.prec[tid];
+    prec = my_prec;
     // An expert whose rows do not lie inside [0, rows) is left out (no unit
     // reads or writes them) and flagged: the epilogue's stores use these rows.
     if (off < 0 || n < 0 || off > p.rows || n > p.rows - off) {
@@ -389,8 +452,11 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
     un.wrow0 = wb * (kSwap ? 128 : 256);
     un.nbox = min(kSwap ? 1 : 2, (p.H - un.wrow0) / kBoxRows);
   }
-  un.flags = kUnitValid | (gu ? kUnitGateUp : 0);
-  un.need = 4 * tiles_of(en.nrows, p) * p.nwb_gu;  // 4 epilogue warps per gate/up unit
+  const bool fma = kSwap && un.prec != MOE_BF16 && en.nrows <= p.fma_rows;
+  un.flags = kUnitValid | (gu ? kUnitGateUp : 0) | (fma ? kUnitFma : 0);
+  // gate/up arrivals: the 4 epilogue warps of a tensor-core unit, or every
+  // dequant warp of a CUDA-core unit (an expert's units are all of one kind)
+  un.need = (fma ? kDequantWarps : 4) * tiles_of(en.nrows, p) * p.nwb_gu;
   return un;
 }
 
@@ -423,9 +489,24 @@ __device__ __forceinline__ void load_scale_box(void* dst, const Params& p, const
   }
 }
 
-// Reduction length of the unit's projection in 64-element k-blocks.
+__device__ __forceinline__ bool unit_fma(const Unit& un) { return (un.flags & kUnitFma) != 0; }
+
+// Operand-ring stages of a unit: one per 64-element k-block, or for a CUDA-core
+// unit one per 128 code bytes of a row (INT4: 256 K-elements, INT8: 128); the
+// last CUDA-core stage may run past K and reads zeros there (TMA fill).
 __device__ __forceinline__ int unit_nkb(const Params& p, const Unit& un) {
-  return (unit_gu(un) ? p.H : p.I) / 64;
+  const int K = unit_gu(un) ? p.H : p.I;
+  if (unit_fma(un)) {
+    const int step = un.prec == MOE_INT4 ? 256 : 128;
+    return (K + step - 1) / step;
+  }
+  return K / 64;
+}
+
+// Bytes a CUDA-core stage receives: codes, X (one or two 128-K boxes) and scales.
+__device__ __forceinline__ uint32_t fma_stage_bytes(int prec) {
+  const uint32_t boxes = prec == MOE_INT4 ? 2u : 1u;
+  return kBoxRows * 128 + boxes * (kFmaRows * 256 + kBoxRows * 2);
 }
 
 __device__ __forceinline__ int ld_acquire(const int* ptr) {
@@ -488,7 +569,10 @@ __device__ void scheduler(const Params& p, const Smem& s) {
     if (u < total) {
       un = decode_unit<kSwap>(p, s, u);
       const ExpertDesc* d = p.descs + un.e;
-      prefetch_tmap(unit_gu(un) ? &d->tm_w13 : &d->tm_w2);
+      if (unit_fma(un))
+        prefetch_tmap(unit_gu(un) ? &d->tm_q13f : &d->tm_q2f);
+      else
+        prefetch_tmap(unit_gu(un) ? &d->tm_w13 : &d->tm_w2);
       if (!unit_gu(un) && !wait_gate_up(p, un, abort_flag)) {
         ok = false;
         break;
@@ -508,25 +592,33 @@ __device__ void scheduler(const Params& p, const Smem& s) {
     FFN_TRACE_SET(tseq, kTrSched, FFN_TRACE_NS());
     ++tseq;
   }
-  if (!ok) give_up(s);
+  if (!ok) give_up(s, 1, tseq);
 }
 
 // ---------------------------------------------------------------- producer --
 // Streams, per k-block, the X tile (one copy) and, for BF16 units, the
 // weight boxes into the operand ring.
 template <bool kSwap>
-__device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const Params& p,
+__device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h,
+                         const CUtensorMap* tm_xf, const CUtensorMap* tm_hf, const Params& p,
                          const Smem& s) {
   volatile int* abort_flag = s.abort_flag;
   const uint32_t ns = p.ns;
   uint32_t st = 0, sph = 0, us = 0, uph = 0;
-  uint32_t issued = 0, issued_par = 0;  // drain bookkeeping
+  // drain bookkeeping: stages with copies issued, whether the last issue was a
+  // CUDA-core one (landing on ffull) and the parity of the phase it completes;
+  // full and ffull each count phases only at their own kind of position
+  uint32_t issued = 0, issued_par = 0, issued_fma = 0, tc_par = 0, fma_par = 0;
   const uint32_t xbytes = (uint32_t)p.xbox_rows * 128;
   bool ok = true;
   int tseq = 0;
   (void)tseq;
   prefetch_tmap(tm_x);
   prefetch_tmap(tm_h);
+  if (kSwap) {
+    prefetch_tmap(tm_xf);
+    prefetch_tmap(tm_hf);
+  }
   for (;;) {
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
       ok = false;
@@ -539,15 +631,22 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
     FFN_TRACE_SET(tseq, kTrProdBeg, FFN_TRACE_NS());
 
     const bool gu = unit_gu(un);
+    const bool fma = kSwap && unit_fma(un);
+    const bool int4 = un.prec == MOE_INT4;
     const ExpertDesc* d = p.descs + un.e;
-    const CUtensorMap* tw = gu ? &d->tm_w13 : &d->tm_w2;
-    const CUtensorMap* tx = gu ? tm_x : tm_h;
+    const CUtensorMap* tw = fma ? (gu ? &d->tm_q13f : &d->tm_q2f) : (gu ? &d->tm_w13 : &d->tm_w2);
+    const CUtensorMap* tsc = gu ? &d->tm_s13f : &d->tm_s2f;
+    const CUtensorMap* tx = fma ? (gu ? tm_xf : tm_hf) : (gu ? tm_x : tm_h);
     const bool bf16 = un.prec == MOE_BF16;
-    if (bf16) tmap_acquire(tw);
+    if (bf16 || fma) tmap_acquire(tw);
+    if (fma) tmap_acquire(tsc);
     if (!gu) fence_proxy_async_global();  // h rows published (scheduler's acquire) -> TMA reads
     const int nkb = unit_nkb(p, un);
-    const uint32_t bytes = xbytes + (bf16 ? (uint32_t)un.nbox * (kBoxRows * 128) : 0u);
+    const uint32_t bytes = fma ? fma_stage_bytes(un.prec)
+                               : xbytes + (bf16 ? (uint32_t)un.nbox * (kBoxRows * 128) : 0u);
     const int reserve_kb = max(0, nkb - (int)ns - 4);
+    long long tr_wait = 0;
+    (void)tr_wait;
     for (int kb = 0; kb < nkb; ++kb) {
       if (kb == reserve_kb) mbar_arrive(s.go);
       const long long c0 = FFN_CLOCK();
@@ -555,31 +654,67 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h, const
         ok = false;
         break;
       }
-      FFN_TRACE_ADD(tseq, kTrProdWait, FFN_CLOCK() - c0);
-      if (!bf16) mbar_arrive(&s.wfree[st]);  // the dequant warps may fill this stage
-      mbar_arrive_expect_tx(&s.full[st], bytes);
-      if (bf16) mbar_arrive_n(&s.full[st], kDequantWarps);  // no dequant at this position
-      tma_load_2d(s.x_st + st * s.xstage, tx, kb * 64, un.row0, &s.full[st]);
-      if (bf16)
-        for (int b = 0; b < un.nbox; ++b)
-          load_weight_box(s.w_st + st * s.wstage + b * (kBoxRows * 128), tw, un, b, kb * 64,
-                          &s.full[st]);
+      tr_wait += FFN_CLOCK() - c0;
+      if (fma) {
+        // CUDA-core position: the data lands on ffull[st], which completes only
+        // at such positions, so the dequant warps count its phases per stage no
+        // matter how many tensor-core positions lie in between (and the MMA
+        // thread, which passes over these positions, counts full's likewise).
+        mbar_arrive_expect_tx(&s.ffull[st], bytes);
+        // 128 code bytes of each of the 128 weight rows, the tile's X rows for
+        // the same K range (one or two 128-element boxes) and the K-groups'
+        // scales; the dequant warps compute the stage on CUDA cores.
+        uint8_t* xdst = s.x_st + st * s.xstage;
+        uint64_t* fb = &s.ffull[st];
+        const int k0 = kb * (int4 ? 256 : 128), g0 = kb * (int4 ? 2 : 1);
+        if (gu)
+          tma_load_3d(s.w_st + st * s.wstage, tw, kb * 128, un.wrow0, 0, fb);
+        else
+          tma_load_2d(s.w_st + st * s.wstage, tw, kb * 128, un.wrow0, fb);
+        tma_load_2d(xdst, tx, k0, un.row0, fb);
+        if (int4) tma_load_2d(xdst + kFmaRows * 256, tx, k0 + 128, un.row0, fb);
+        if (gu)
+          tma_load_3d(xdst + kFmaXBytes, tsc, un.wrow0, 0, g0, fb);
+        else
+          tma_load_2d(xdst + kFmaXBytes, tsc, un.wrow0, g0, fb);
+        issued_fma |= 1u << st;
+        issued_par = (issued_par & ~(1u << st)) | (((fma_par >> st) & 1u) << st);
+        fma_par ^= 1u << st;
+      } else {
+        // INT8/INT4 tensor-core position: the dequant warps may fill this
+        // stage.  They pass over BF16 units without waiting and may be ring
+        // revolutions ahead; wfree, complete only at these positions, tells
+        // them the producer has reached it.
+        if (!bf16) mbar_arrive(&s.wfree[st]);
+        mbar_arrive_expect_tx(&s.full[st], bytes);
+        if (bf16) mbar_arrive_n(&s.full[st], kDequantWarps);  // no dequant at this position
+        tma_load_2d(s.x_st + st * s.xstage, tx, kb * 64, un.row0, &s.full[st]);
+        if (bf16)
+          for (int b = 0; b < un.nbox; ++b)
+            load_weight_box(s.w_st + st * s.wstage + b * (kBoxRows * 128), tw, un, b, kb * 64,
+                            &s.full[st]);
+        issued_fma &= ~(1u << st);
+        issued_par = (issued_par & ~(1u << st)) | (((tc_par >> st) & 1u) << st);
+        tc_par ^= 1u << st;
+      }
       issued |= 1u << st;
-      issued_par = (issued_par & ~(1u << st)) | (sph << st);
       advance(st, sph, ns);
     }
     if (!ok) break;
     FFN_TRACE_SET(tseq, kTrProdEnd, FFN_TRACE_NS());
+    FFN_TRACE_SET(tseq, kTrProdWait, tr_wait);
     ++tseq;
   }
   if (!ok) {
-    give_up(s);
+    give_up(s, 2, tseq);
     // Let copies already in flight land before the CTA's shared memory goes
     // away.  The full barrier of an INT8/INT4 position also counts dequant
     // arrivals, which may never come once the CTA gives up, so each wait is
     // cut short after about a millisecond (copies land within microseconds).
     for (uint32_t i = 0; i < ns; ++i)
-      if (issued & (1u << i)) mbar_wait(&s.full[i], (issued_par >> i) & 1u, nullptr, kDrainCycles);
+      if (issued & (1u << i))
+        mbar_wait((issued_fma >> i) & 1u ? &s.ffull[i] : &s.full[i], (issued_par >> i) & 1u,
+                  nullptr, kDrainCycles);
   }
 }
 
@@ -605,7 +740,7 @@ __device__ void code_producer(const Params& p, const Smem& s) {
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
     ++tseq;
-    if (un.prec == MOE_BF16) continue;
+    if (un.prec == MOE_BF16 || unit_fma(un)) continue;
     const bool gu = unit_gu(un);
     const ExpertDesc* d = p.descs + un.e;
     const CUtensorMap* tw = gu ? &d->tm_w13 : &d->tm_w2;
@@ -613,13 +748,15 @@ __device__ void code_producer(const Params& p, const Smem& s) {
     prefetch_tmap(tw);
     const int nkb = unit_nkb(p, un);
     const bool int4 = un.prec == MOE_INT4;
+    long long tr_wait = 0;
+    (void)tr_wait;
     for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
       const long long c0 = FFN_CLOCK();
       if (!mbar_wait(&s.qempty[q], qph ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
-      FFN_TRACE_ADD(tseq, kTrCodeWait, FFN_CLOCK() - c0);
+      tr_wait += FFN_CLOCK() - c0;
       mbar_arrive_expect_tx(&s.qfull[q], (uint32_t)un.nbox * (kBoxRows * 64 + kBoxRows * 2));
       const int kc = int4 ? (kb >> 1) * 64 : kb * 64;  // byte column of the codes
       const int g = kb >> 1;                            // K-group of the scales
@@ -632,9 +769,10 @@ __device__ void code_producer(const Params& p, const Smem& s) {
       advance(q, qph, nq);
     }
     if (!ok) break;
+    FFN_TRACE_SET(tseq, kTrCodeWait, tr_wait);
   }
   if (!ok) {
-    give_up(s);
+    give_up(s, 3, tseq);
     for (uint32_t i = 0; i < nq; ++i)
       if (qissued & (1u << i)) mbar_wait(&s.qfull[i], (qissued_par >> i) & 1u);
   }
@@ -677,6 +815,7 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
   const uint64_t xdesc0 = smem_desc_sw128(smem_u32(s.x_st));
   const uint32_t wstep = s.wstage >> 4, xstep = s.xstage >> 4;
   uint32_t st = 0, sph = 0, us = 0, uph = 0, abuf = 0;
+  uint32_t tph = 0;  // full phase bit per stage: it only advances at tensor-core positions
   uint32_t aph[2] = {0, 0};
   bool ok = true;
   int tseq = 0;
@@ -691,6 +830,11 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
     const int nkb = unit_nkb(p, un);
+    if (kSwap && unit_fma(un)) {  // computed and freed by the dequant warps
+      for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
+      ++tseq;
+      continue;
+    }
     if (!mbar_wait(&s.accempty[abuf], aph[abuf] ^ 1u, abort_flag)) {
       ok = false;
       break;
@@ -702,13 +846,18 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
     const uint32_t idesc = idesc_bf16_f32(128, n);
     const bool quant = un.prec != MOE_BF16;
     const bool a_in_tmem = kSwap && quant;  // dequantised weights live in TMEM
+    long long tr_wait = 0, tr_issue = 0;
+    (void)tr_wait;
+    (void)tr_issue;
     for (int kb = 0; kb < nkb; ++kb) {
       const long long c0 = FFN_CLOCK();
-      if (!mbar_wait(&s.full[st], sph, abort_flag)) {  // X landed, weights in place
+      if (!mbar_wait(&s.full[st], (tph >> st) & 1u, abort_flag)) {  // X landed, weights in place
         ok = false;
         break;
       }
-      FFN_TRACE_ADD(tseq, kTrMmaWait, FFN_CLOCK() - c0);
+      tph ^= 1u << st;
+      const long long c1 = FFN_CLOCK();
+      tr_wait += c1 - c0;
       tc_fence_after();
       const uint64_t xd = xdesc0 + st * xstep, wd = wdesc0 + st * wstep;
       const uint32_t acc0 = kb != 0;
@@ -720,15 +869,18 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
         mma_kblock_ss(d_tmem, xd, wd, idesc, acc0);
       mma_commit(&s.empty[st]);
       advance(st, sph, ns);
+      tr_issue += FFN_CLOCK() - c1;
     }
     if (!ok) break;
     mma_commit(&s.accfull[abuf]);
     FFN_TRACE_SET(tseq, kTrMmaEnd, FFN_TRACE_NS());
+    FFN_TRACE_SET(tseq, kTrMmaWait, tr_wait);
+    FFN_TRACE_SET(tseq, kTrMmaIssue, tr_issue);
     ++tseq;
     aph[abuf] ^= 1u;
     abuf ^= 1u;
   }
-  if (!ok) give_up(s);
+  if (!ok) give_up(s, 4, tseq);
   // All issued MMAs must finish before TMEM is released.
   mma_commit(s.mmadone);
   mbar_wait(s.mmadone, 0);
@@ -780,6 +932,240 @@ __device__ __forceinline__ uint64_t f32x2(float v) {
   return r;
 }
 
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+// Gate/up results: once this warp's h stores are done, publish them to the
+// down units of the expert (release counter; the proxy fence orders the
+// generic-proxy stores before any TMA read that the counter enables).
+__device__ __forceinline__ void publish_expert(const Params& p, int e, int lane) {
+  fence_proxy_async_global();
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) red_release_add(p.done + e, 1);
+}
+
+__device__ __forceinline__ void publish_rows(const Params& p, const Unit& un, int lane) {
+  publish_expert(p, un.e, lane);
+}
+
+// ------------------------------------------------------- CUDA-core units --
+// A stage holds 128 weight rows x 128 code bytes ([2][64][128] for gate/up:
+// gate rows, then the same up rows), X as [box][kFmaRows][128] bf16 and the
+// scales as [group][128 rows] fp16.  Dequant thread ft (0..255) owns K-chunk
+// c = ft % 16 of every row 16 j + ft / 16 (j = 0..7): 8 code bytes, i.e. 16
+// INT4 or 8 INT8 elements; a warp's code loads cover 256 contiguous bytes.  Its
+// X values (fp32 pairs) are loaded once per stage and serve all 8 rows.  Rows
+// j and j + 4 of a gate/up unit are a gate row and its up row, so the SwiGLU
+// needs no exchange.  Dot products are exact-product fp32 sums:
+//   INT4: a code u becomes the fp32 value 128 + u (u placed in bits 16..19 of
+//     128.0, one prmt); sum_k (128 + u_k) x_k - 136 sum_k x_k = sum_k q_k x_k
+//     with q = u - 8, every product exact (8 x 8 significant bits);
+//   INT8: 32768 + (q + 128) (the byte in bits 8..15 of 2^15), minus 32896
+//     exactly, then exact products.
+// The K-group's scale multiplies each partial sum (fp32), the 16 lanes of a
+// row are summed at the end of the unit, and the results are rounded to bf16
+// once (h = silu(g) * u for gate/up, y for down).
+
+__device__ __forceinline__ uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ float hsum2(uint64_t v) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  return __uint_as_float(lo) + __uint_as_float(hi);
+}
+
+// bf16x2 word (element 2i in the low half) -> fp32 pair, exactly.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  return pack_f32x2(w << 16, w & 0xFFFF0000u);
+}
+
+// Byte b of a (an INT4 nibble 0..15) -> fp32 128 + nibble.
+__device__ __forceinline__ uint32_t nib_f32(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0x43000000, %2;" : "=r"(d) : "r"(a), "r"(0x7044u | (b << 8)));
+  return d;
+}
+
+template <int N, bool kInt4>
+__device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const Unit& un, int ft,
+                                         uint32_t& st, uint32_t& sph, uint32_t& ffph,
+                                         uint32_t& fdph, int& pub_e, long long* tr) {
+  long long& tr_wait = tr[0];
+  long long& tr_conv = tr[1];
+  long long& tr_sync = tr[2];
+  long long& tr_out = tr[3];
+  long long& tr_pub = tr[4];
+  (void)tr_sync;
+  (void)tr_out;
+  (void)tr_pub;
+  volatile int* abort_flag = s.abort_flag;
+  const uint32_t ns = p.ns;
+  const int lane = threadIdx.x & 31;
+  const int c = ft & 15, rsub = ft >> 4;
+  constexpr int kPairs = kInt4 ? 8 : 4;  // element pairs of a lane's chunk
+  const int nkb = unit_nkb(p, un);
+  float acc[8][N];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int n = 0; n < N; ++n) acc[j][n] = 0.0f;
+  const uint64_t off2 = pack_f32x2(__float_as_uint(-32896.0f), __float_as_uint(-32896.0f));
+  const uint64_t one2 = pack_f32x2(__float_as_uint(1.0f), __float_as_uint(1.0f));
+  (void)off2;
+  (void)one2;
+  for (int kb = 0; kb < nkb; ++kb) {
+    // ffull counts phases at CUDA-core positions only (bits in ffph, per stage)
+    const long long c0 = FFN_CLOCK();
+    if (!mbar_wait(&s.ffull[st], (ffph >> st) & 1u, abort_flag)) return false;
+    ffph ^= 1u << st;
+    const long long c1 = FFN_CLOCK();
+    tr_wait += c1 - c0;
+    const uint8_t* xs = s.x_st + st * s.xstage;
+    const uint8_t* codes = s.w_st + st * s.wstage;
+    // X of this lane's chunk, fp32 pairs, and (INT4) its per-token sum
+    uint64_t xv[N][kPairs];
+    float sx[N];
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+      if (kInt4) {
+        const uint4* src = reinterpret_cast<const uint4*>(xs + (c >> 3) * (kFmaRows * 256) +
+                                                          n * 256 + (c & 7) * 32);
+        const uint4 a = src[0], b = src[1];
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        float t = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          xv[n][i] = bf16x2_to_f32x2(w[i]);
+          t += hsum2(xv[n][i]);
+        }
+        sx[n] = t;
+      } else {
+        const uint4 a = *reinterpret_cast<const uint4*>(xs + n * 256 + c * 16);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[n][i % kPairs] = bf16x2_to_f32x2(w[i]);
+        sx[n] = 0.0f;
+      }
+    }
+    const __half* sc = reinterpret_cast<const __half*>(xs + kFmaXBytes) + (kInt4 ? (c >> 3) * 128 : 0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = 16 * j + rsub;
+      const uint2 w = *reinterpret_cast<const uint2*>(codes + r * 128 + c * 8);
+      const float sr = __half2float(sc[r]);
+      uint64_t d[N];
+#pragma unroll
+      for (int n = 0; n < N; ++n) d[n] = 0;
+      if (kInt4) {
+        const uint32_t wd[2] = {w.x, w.y};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t lo = wd[h] & 0x0F0F0F0Fu, hi = (wd[h] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const uint64_t m = pack_f32x2(nib_f32(lo, b), nib_f32(hi, b));  // elements 2i, 2i+1
+#pragma unroll
+            for (int n = 0; n < N; ++n) d[n] = ffma2(m, xv[n][4 * h + b], d[n]);
+          }
+        }
+#pragma unroll
+        for (int n = 0; n < N; ++n)
+          acc[j][n] = fmaf(sr, fmaf(-136.0f, sx[n], hsum2(d[n])), acc[j][n]);
+      } else {
+        const uint32_t wd[2] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u};
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const uint64_t m = pack_f32x2(place_byte(wd[h], sel_byte(2 * b)),
+                                          place_byte(wd[h], sel_byte(2 * b + 1)));
+            const uint64_t q = ffma2(m, one2, off2);  // exact: the integer q of each code
+#pragma unroll
+            for (int n = 0; n < N; ++n) d[n] = ffma2(q, xv[n][(2 * h + b) % kPairs], d[n]);
+          }
+#pragma unroll
+        for (int n = 0; n < N; ++n) acc[j][n] = fmaf(sr, hsum2(d[n]), acc[j][n]);
+      }
+    }
+    tr_conv += FFN_CLOCK() - c1;
+    // Every dequant warp is done with the stage: thread 0 forwards the eight
+    // arrivals to the stage's empty barrier (the producer's refill condition).
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.fdone[st]);
+    if (ft == 0) {
+      const long long c2 = FFN_CLOCK();
+      if (!mbar_wait(&s.fdone[st], (fdph >> st) & 1u, abort_flag)) return false;
+      tr_sync += FFN_CLOCK() - c2;
+      mbar_arrive(&s.empty[st]);
+    }
+    fdph ^= 1u << st;
+    advance(st, sph, ns);
+    // the previous gate/up unit's h rows, stored a stage ago: publishing them
+    // now costs little (the fence no longer waits for stores in flight)
+    if (pub_e >= 0) {
+      publish_expert(p, pub_e, lane);
+      pub_e = -1;
+    }
+  }
+  const long long c3 = FFN_CLOCK();
+  // sum the 16 lanes (K-chunks) of each row; every lane ends with the totals
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+      float v = acc[j][n];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      acc[j][n] = v;
+    }
+  if (unit_gu(un)) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int n = 0; n < N; ++n)
+        if (c == n && n < un.nrows)
+          p.h[(size_t)(un.row0 + n) * p.I + un.wrow0 + 16 * j + rsub] =
+              __float2bfloat16_rn(silu_mul(acc[j][n], acc[j + 4][n]));
+    pub_e = un.e;  // published by the caller later (deferred publication)
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int n = 0; n < N; ++n)
+        if (c == n && n < un.nrows)
+          p.y[(size_t)(un.row0 + n) * p.H + un.wrow0 + 16 * j + rsub] =
+              __float2bfloat16_rn(acc[j][n]);
+  }
+  tr_out += FFN_CLOCK() - c3;
+  return true;
+}
+
+template <bool kInt4>
+__device__ bool fma_dispatch(const Params& p, const Smem& s, const Unit& un, int ft, uint32_t& st,
+                             uint32_t& sph, uint32_t& ffph, uint32_t& fdph, int& pub_e,
+                             long long* tr) {
+  static_assert(kFmaRows >= 1 && kFmaRows <= 4, "CUDA-core tiles of 1 to 4 rows");
+  if (kFmaRows >= 4 && un.nrows == 4)
+    return fma_unit<4, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+  if (kFmaRows >= 3 && un.nrows == 3)
+    return fma_unit<3, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+  if (kFmaRows >= 2 && un.nrows == 2)
+    return fma_unit<2, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+  return fma_unit<1, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+}
+
 // One staging slot holds an INT4 group (128 K-elements = two k-blocks) or an
 // INT8 k-block (64 K-elements) for the unit's weight rows, 64 bytes per row.
 // Work item = 16 bytes of codes of one row: INT4 -> 32 elements (4 output
@@ -803,13 +1189,25 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
   const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + p.a_col;
   const uint32_t ns = p.ns, nq = p.nq;
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
-  uint32_t fph = 0;  // wfree phase bit per stage: it only advances on INT8/INT4 positions
+  uint32_t fph = 0;   // wfree phase bit per stage: INT8/INT4 tensor-core positions only
+  uint32_t ffph = 0;  // ffull phase bit per stage: CUDA-core positions only
+  uint32_t fdph = 0;  // fdone phase bit per stage: CUDA-core positions only
+  const int ft = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // warps 2, 3, 8 .. 13
+  // A CUDA-core gate/up unit's h rows are published (fence + release add) one
+  // stage into the next CUDA-core unit, when their stores have landed -- and
+  // always before this warp could block on anything a down unit's wait could
+  // hold up: the unit ring, or an INT8/INT4 tensor-core unit.
+  int pub_e = -1;
   bool ok = true;
   int tseq = -1;
   const bool tracer = warp == 2 && lane == 0;
   (void)tseq;
   (void)tracer;
   for (;;) {
+    if (pub_e >= 0 && !mbar_try_wait(&s.ufull[us], uph)) {
+      publish_expert(p, pub_e, lane);
+      pub_e = -1;
+    }
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
       ok = false;
       break;
@@ -821,13 +1219,38 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
     if (!(un.flags & kUnitValid)) break;
     ++tseq;
     const int nkb = unit_nkb(p, un);
+    if (pub_e >= 0 && !unit_fma(un)) {
+      publish_expert(p, pub_e, lane);
+      pub_e = -1;
+    }
     if (un.prec == MOE_BF16) {
       for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
       continue;
     }
     if (tracer) FFN_TRACE_SET(tseq, kTrDqBeg, FFN_TRACE_NS());
+    if (unit_fma(un)) {
+      long long tr[5] = {0, 0, 0, 0, 0};
+      ok = un.prec == MOE_INT4
+               ? fma_dispatch<true>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr)
+               : fma_dispatch<false>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+      if (!ok) break;
+      if (tracer) {
+        FFN_TRACE_SET(tseq, kTrDqEnd, FFN_TRACE_NS());
+        FFN_TRACE_SET(tseq, kTrDqWaitQ, tr[0]);
+        FFN_TRACE_SET(tseq, kTrDqConv, tr[1]);
+        FFN_TRACE_SET(tseq, kTrDqWaitW, tr[2]);
+        FFN_TRACE_SET(tseq, kTrDqStore, tr[3]);
+        FFN_TRACE_SET(tseq, kTrPublish, tr[4]);
+      }
+      continue;
+    }
     const bool int4 = un.prec == MOE_INT4;
     const float off = int4 ? 32776.0f : 32896.0f;  // 2^15 + 8, 2^15 + 128
+    long long tr_wq = 0, tr_ww = 0, tr_conv = 0, tr_store = 0;
+    (void)tr_wq;
+    (void)tr_ww;
+    (void)tr_conv;
+    (void)tr_store;
     for (int kb = 0; kb < nkb; kb += int4 ? 2 : 1) {
       const uint32_t st0 = st;
       advance(st, sph, ns);
@@ -844,10 +1267,9 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
         ok = false;
         break;
       }
-      if (tracer) {
-        FFN_TRACE_ADD(tseq, kTrDqWaitQ, tq1 - tq0);
-        FFN_TRACE_ADD(tseq, kTrDqWaitW, FFN_CLOCK() - tq1);
-      }
+      const long long tq2 = FFN_CLOCK();
+      tr_wq += tq1 - tq0;
+      tr_ww += tq2 - tq1;
       fph ^= (1u << st0) | (int4 ? 1u << st1 : 0u);
       tc_fence_after();
       const uint4* src = reinterpret_cast<const uint4*>(s.q_st + q * s.qslot + r * 64 + half * 32);
@@ -863,6 +1285,7 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
 #pragma unroll
           for (int b = 0; b < 4; ++b) v[4 * j + b] = deq2(lo, sel_byte(b), hi, sel_byte(b), s2, k2);
         }
+        tr_conv += FFN_CLOCK() - tq2;
         tmem_st32(lane_addr + (half ? st1 : st0) * 32, v);
       } else {
         uint32_t v[16];  // word j = elements 4 j .. 4 j + 3 -> columns 2 j, 2 j + 1
@@ -872,8 +1295,10 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
           v[2 * j] = deq2(a, sel_byte(0), a, sel_byte(1), s2, k2);
           v[2 * j + 1] = deq2(a, sel_byte(2), a, sel_byte(3), s2, k2);
         }
+        tr_conv += FFN_CLOCK() - tq2;
         tmem_st16(lane_addr + st0 * 32 + half * 16, v);
       }
+      const long long tq3 = FFN_CLOCK();
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -883,11 +1308,19 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
         mbar_arrive(&s.qempty[q]);
       }
       advance(q, qph, nq);
+      tr_store += FFN_CLOCK() - tq3;
     }
     if (!ok) break;
-    if (tracer) FFN_TRACE_SET(tseq, kTrDqEnd, FFN_TRACE_NS());
+    if (tracer) {
+      FFN_TRACE_SET(tseq, kTrDqEnd, FFN_TRACE_NS());
+      FFN_TRACE_SET(tseq, kTrDqWaitQ, tr_wq);
+      FFN_TRACE_SET(tseq, kTrDqWaitW, tr_ww);
+      FFN_TRACE_SET(tseq, kTrDqConv, tr_conv);
+      FFN_TRACE_SET(tseq, kTrDqStore, tr_store);
+    }
   }
-  if (!ok) give_up(s);
+  if (pub_e >= 0) publish_expert(p, pub_e, lane);
+  if (!ok) give_up(s, 5, tseq);
 }
 
 __device__ void dequant(const Params& p, const Smem& s, int dtid) {
@@ -993,17 +1426,6 @@ __device__ void dequant(const Params& p, const Smem& s, int dtid) {
 }
 
 // ---------------------------------------------------------------- epilogue --
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
-
-// Gate/up epilogue: once this warp's h stores are done, publish them to the
-// down units of the expert (release counter; the proxy fence orders the
-// generic-proxy stores before any TMA read that the counter enables).
-__device__ __forceinline__ void publish_rows(const Params& p, const Unit& un, int lane) {
-  fence_proxy_async_global();
-  __threadfence();
-  __syncwarp();
-  if (lane == 0) red_release_add(p.done + un.e, 1);
-}
 
 template <bool kSwap>
 __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
@@ -1029,6 +1451,10 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
     const bool gu = unit_gu(un);
+    if (kSwap && unit_fma(un)) {  // the dequant warps store and publish its rows
+      ++tseq;
+      continue;
+    }
     if (!mbar_wait(&s.accfull[ebuf], eph[ebuf], abort_flag)) {
       ok = false;
       break;
@@ -1119,21 +1545,28 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.accempty[ebuf]);
+    const long long cp = FFN_CLOCK();
     if (gu) publish_rows(p, un, lane);
-    if (tracer) FFN_TRACE_SET(tseq, kTrEpiEnd, FFN_TRACE_NS());
+    if (tracer) {
+      FFN_TRACE_SET(tseq, kTrEpiEnd, FFN_TRACE_NS());
+      FFN_TRACE_SET(tseq, kTrPublish, FFN_CLOCK() - cp);
+    }
     ++tseq;
     eph[ebuf] ^= 1u;
     ebuf ^= 1u;
   }
-  if (!ok) give_up(s);
+  if (!ok) give_up(s, 6, tseq);
 }
 
 // ------------------------------------------------------------------ kernel --
 template <bool kSwap>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_ffn_kernel(const __grid_constant__ CUtensorMap tm_x,
-                       const __grid_constant__ CUtensorMap tm_h, const Params p) {
+                       const __grid_constant__ CUtensorMap tm_h,
+                       const __grid_constant__ CUtensorMap tm_xf,
+                       const __grid_constant__ CUtensorMap tm_hf, const Params p) {
   extern __shared__ uint8_t ffn_smem_raw[];
+  FFN_KSTAMP(0);
   const Smem s = carve(ffn_smem_raw, p, kSwap);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -1145,8 +1578,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // producer's arrive.expect_tx, then one arrival per dequant warp (INT8/INT4
       // positions) or kDequantWarps more from the producer (BF16 positions)
       mbar_init(&s.full[i], 1 + kDequantWarps);
-      mbar_init(&s.empty[i], 1);               // tcgen05.commit
-      mbar_init(&s.wfree[i], 1);               // producer, at INT8/INT4 positions
+      mbar_init(&s.empty[i], 1);               // tcgen05.commit, or dequant thread 0 (CUDA-core)
+      mbar_init(&s.wfree[i], 1);               // producer, at INT8/INT4 tensor-core positions
+      mbar_init(&s.fdone[i], kDequantWarps);   // each dequant warp, at CUDA-core positions
+      mbar_init(&s.ffull[i], 1);               // producer's expect_tx, at CUDA-core positions
     } else if (i >= kMaxNS && i < kMaxNS + kMaxNQ) {
       mbar_init(&s.qfull[i - kMaxNS], 1);
       mbar_init(&s.qempty[i - kMaxNS], kDequantWarps);
@@ -1170,16 +1605,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(s.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  const int my_prec = (int)threadIdx.x < p.E ? p.prec[threadIdx.x] : -1;
   pdl_launch_dependents();
+  FFN_KSTAMP(1);
   pdl_wait();           // inputs of the previous kernels are complete from here on
-  build_entries<kSwap>(p, s);  // contains a __syncthreads
+  build_entries<kSwap>(p, s, my_prec);  // contains a __syncthreads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  FFN_KSTAMP(2);
   const uint32_t tmem = *s.tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) producer<kSwap>(&tm_x, &tm_h, p, s);
+    if (lane == 0) producer<kSwap>(&tm_x, &tm_h, &tm_xf, &tm_hf, p, s);
   } else if (warp == 1) {
     if (lane == 0) mma_issuer<kSwap>(p, s, tmem);
   } else if (warp >= 4 && warp < 8) {
@@ -1197,10 +1635,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  FFN_KSTAMP(3);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  FFN_KSTAMP(4);
 }
 
 // Stream-ordered install of one expert descriptor (a by-value kernel argument,
@@ -1209,8 +1649,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void write_desc_kernel(ExpertDesc* dst, int* prec_dst,
                                   const __grid_constant__ ExpertDesc d) {
   const int i = threadIdx.x;
-  if (i < (int)(sizeof(ExpertDesc) / 16))
-    reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(&d)[i];
+  for (int v = i; v < (int)(sizeof(ExpertDesc) / 16); v += blockDim.x)
+    reinterpret_cast<uint4*>(dst)[v] = reinterpret_cast<const uint4*>(&d)[v];
   if (i == 0) *prec_dst = d.prec;
   tmap_release();
 }

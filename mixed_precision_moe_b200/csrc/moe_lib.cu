@@ -116,6 +116,12 @@ int encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int e
 //   w2 [H][K] as a 2-D map with box 128 x 64.
 // BF16 values land in the 128-byte-swizzled layout the MMA reads; INT8/INT4
 // codes (64 bytes of a row per box) are staged unswizzled and dequantised.
+// INT8/INT4 experts also get the maps of the CUDA-core path (layers with H and I
+// of at least 256): codes in 128-byte K boxes (128 rows: 64 gate + 64 up rows,
+// or 128 down rows) and the fp16 scales of one stage's K-groups (INT4: two,
+// INT8: one) for the same rows, the gate/up scales viewed as [G][2][I].
+bool fma_capable(int H, int I) { return H >= 256 && I >= 256; }
+
 int encode_weights(moe::ffn::ExpertDesc* d, const moe_expert_weights* w, int prec, int H, int I) {
   const bool bf16 = prec == MOE_BF16;
   const CUtensorMapDataType t = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -124,7 +130,20 @@ int encode_weights(moe::ffn::ExpertDesc* d, const moe_expert_weights* w, int pre
   const int cols13 = prec == MOE_INT4 ? H / 2 : H, cols2 = prec == MOE_INT4 ? I / 2 : I;
   int rc = encode_3d(&d->tm_w13, w->w13, t, es, 2, I, cols13, 2, 64, 64, swz);
   if (rc != MOE_OK) return rc;
-  return encode_2d(&d->tm_w2, w->w2, t, es, H, cols2, 128, 64, swz);
+  rc = encode_2d(&d->tm_w2, w->w2, t, es, H, cols2, 128, 64, swz);
+  if (rc != MOE_OK || bf16 || !fma_capable(H, I)) return rc;
+  const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  const uint32_t gs = prec == MOE_INT4 ? 2 : 1;  // K-groups per CUDA-core stage
+  rc = encode_3d(&d->tm_q13f, w->w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 2, I, cols13, 2, 64, 128,
+                 none);
+  if (rc != MOE_OK) return rc;
+  rc = encode_2d(&d->tm_q2f, w->w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H, cols2, 128, 128, none);
+  if (rc != MOE_OK) return rc;
+  rc = encode_3d(&d->tm_s13f, w->s13, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, H / 128, 2, I, gs, 2, 64,
+                 none);
+  if (rc != MOE_OK) return rc;
+  return encode_2d(&d->tm_s2f, w->s2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, I / 128, H, gs, 128,
+                   none);
 }
 
 // Launch with programmatic stream serialization: the kernel may be scheduled
@@ -181,6 +200,22 @@ int moe_ffn_trace_reset(void) {
   void* addr = nullptr;
   MOE_CUDA_TRY(cudaGetSymbolAddress(&addr, moe::ffn::g_ffn_trace));
   MOE_CUDA_TRY(cudaMemset(addr, 0, sizeof(moe::ffn::g_ffn_trace)));
+  return ok();
+}
+
+int moe_ffn_giveup_read(int* host_dst, size_t bytes) {
+  MOE_CHECK(host_dst != nullptr && bytes <= sizeof(moe::ffn::g_ffn_giveup), MOE_ERR_INVALID_ARG,
+            "bad buffer");
+  MOE_CUDA_TRY(cudaMemcpyFromSymbol(host_dst, moe::ffn::g_ffn_giveup, bytes));
+  static const int zero[moe::ffn::kTraceCtas * 4] = {};
+  MOE_CUDA_TRY(cudaMemcpyToSymbol(moe::ffn::g_ffn_giveup, zero, sizeof zero));
+  return ok();
+}
+
+int moe_ffn_kstamp_read(long long* host_dst, size_t bytes) {
+  MOE_CHECK(host_dst != nullptr && bytes <= sizeof(moe::ffn::g_ffn_kstamp), MOE_ERR_INVALID_ARG,
+            "bad buffer");
+  MOE_CUDA_TRY(cudaMemcpyFromSymbol(host_dst, moe::ffn::g_ffn_kstamp, bytes));
   return ok();
 }
 
@@ -481,27 +516,39 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
   const int smem = (int)smem_map(swap, ns, nq, xrows, L->E).total;
   MOE_CHECK(smem <= kSmemLimit, MOE_ERR_UNSUPPORTED, "shared memory plan does not fit");
 
-  CUtensorMap tm_x, tm_h;
+  CUtensorMap tm_x, tm_h, tm_xf, tm_hf;
   rc = encode_2d(&tm_x, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->H, xbox, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
+                 CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != MOE_OK) return rc;
   rc = encode_2d(&tm_h, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->I, xbox, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != MOE_OK) return rc;
+  // CUDA-core units (swap mode): X rows of a tile in 128-element boxes, unswizzled
+  const int fma_rows = swap && fma_capable(L->H, L->I) ? kFmaRows : 0;
+  memset(&tm_xf, 0, sizeof tm_xf);
+  memset(&tm_hf, 0, sizeof tm_hf);
+  if (fma_rows > 0) {
+    rc = encode_2d(&tm_xf, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->H, kFmaRows, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc != MOE_OK) return rc;
+    rc = encode_2d(&tm_hf, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, L->I, kFmaRows, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc != MOE_OK) return rc;
+  }
 
   Params prm{L->d_descs, L->d_prec, expert_offsets, h, static_cast<__nv_bfloat16*>(y_perm),
              counters, counters + 16, rows, L->E, L->H, L->I,
              swap ? L->I / 64 : L->I / 128, swap ? L->H / 128 : (L->H + 255) / 256,
-             xbox, xrows, ns, nq, acc_stride, a_col};
+             xbox, xrows, ns, nq, acc_stride, a_col, fma_rows};
 
   rc = set_ffn_attributes(dev);
   if (rc != MOE_OK) return rc;
   if (swap)
     MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<true>, dim3(grid), dim3(kThreads), smem, s, tm_x,
-                            tm_h, prm));
+                            tm_h, tm_xf, tm_hf, prm));
   else
     MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<false>, dim3(grid), dim3(kThreads), smem, s, tm_x,
-                            tm_h, prm));
+                            tm_h, tm_xf, tm_hf, prm));
   return ok();
 }
 }  // namespace

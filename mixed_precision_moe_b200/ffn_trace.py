@@ -26,7 +26,7 @@ import numpy as np
 
 FIELDS = ["unit", "kind", "sched", "prod_beg", "prod_end", "prod_wait", "code_wait", "mma_beg",
           "mma_end", "mma_wait", "dq_beg", "dq_end", "dq_wait_q", "dq_wait_w", "epi_beg",
-          "epi_end"]
+          "epi_end", "mma_issue", "dq_conv", "dq_store", "publish"]
 F = {n: i for i, n in enumerate(FIELDS)}
 CTAS, UNITS = 160, 96
 
@@ -41,8 +41,8 @@ def summarise(rec: np.ndarray, sm_ghz: float) -> dict:
     valid = rec[:, :, F["sched"]] != 0
     rows = rec[valid]
     t0 = rows[:, F["sched"]].min()
-    out = {"units": int(len(rows)),
-           "kernel_span_us": float((rows[:, F["epi_end"]].max() - t0) / 1e3),
+    last = max(rows[:, F["epi_end"]].max(), rows[:, F["dq_end"]].max())
+    out = {"units": int(len(rows)), "kernel_span_us": float((last - t0) / 1e3),
            "sm_ghz_assumed": sm_ghz}
     cyc = 1e-3 / sm_ghz   # cycles -> us
     groups: dict = {}
@@ -52,21 +52,23 @@ def summarise(rec: np.ndarray, sm_ghz: float) -> dict:
     for key, g in sorted(groups.items()):
         g = np.array(g)
         o = {"n": int(len(g)), "mean_rows": float(np.mean((g[:, F["kind"]] >> 16) & 0xFF))}
-        o["prod_us"] = float(np.mean(g[:, F["prod_end"]] - g[:, F["prod_beg"]]) / 1e3)
-        o["mma_us"] = float(np.mean(g[:, F["mma_end"]] - g[:, F["mma_beg"]]) / 1e3)
-        o["epi_us"] = float(np.mean(g[:, F["epi_end"]] - g[:, F["epi_beg"]]) / 1e3)
-        o["life_us"] = float(np.mean(g[:, F["epi_end"]] - g[:, F["prod_beg"]]) / 1e3)
-        for w in ("prod_wait", "code_wait", "mma_wait", "dq_wait_q", "dq_wait_w"):
+        def span(a, b):   # mean over the units the role stamped (CUDA-core units skip some)
+            m = g[:, F[a]] != 0
+            return float(np.mean(g[m, F[b]] - g[m, F[a]]) / 1e3) if m.any() else None
+        o["prod_us"] = span("prod_beg", "prod_end")
+        o["mma_us"] = span("mma_beg", "mma_end")
+        o["epi_us"] = span("epi_beg", "epi_end")
+        o["dq_span_us"] = span("dq_beg", "dq_end")
+        for w in ("prod_wait", "code_wait", "mma_wait", "mma_issue", "dq_wait_q", "dq_wait_w",
+                  "dq_conv", "dq_store", "publish"):
             o[w + "_us"] = float(np.mean(g[:, F[w]]) * cyc)
-        dq = g[g[:, F["dq_beg"]] != 0]
-        if len(dq):
-            o["dq_us"] = float(np.mean(dq[:, F["dq_end"]] - dq[:, F["dq_beg"]]) / 1e3)
         out[key] = o
     spans, busy = [], []
     for c in range(rec.shape[0]):
         r = rec[c][rec[c][:, F["sched"]] != 0]
         if len(r):
-            spans.append((r[:, F["epi_end"]].max() - r[:, F["prod_beg"]].min()) / 1e3)
+            end = max(r[:, F["epi_end"]].max(), r[:, F["dq_end"]].max())
+            spans.append((end - r[:, F["prod_beg"]].min()) / 1e3)
             busy.append((r[:, F["prod_beg"]].min() - t0) / 1e3)
     out["cta_span_us"] = {"min": float(np.min(spans)), "mean": float(np.mean(spans)),
                           "max": float(np.max(spans))}
@@ -92,7 +94,26 @@ def build_workload(name, device):
     import bench
     from mixed_precision_moe_b200 import binding as B
     from mixed_precision_moe_b200 import synth
-    if name.startswith("decode"):
+    if name == "stack":   # layer 0 of the Qwen3-80B-scale stack, step 0 (experts drawn on the device)
+        S = synth.STACK
+        T, E = S["T"], S["E"]
+        gen = torch.Generator(device=device)
+        gen.manual_seed(S["seed"])
+        layer = B.MoELayer(S["H"], S["I"], E, S["k"])
+        hot = set(np.argsort(synth.stack_ranks(0, 0), kind="stable")[:S["n_hot"]].tolist())
+        for e in range(E):
+            w13 = bench.device_master(2 * S["I"], S["H"], gen, device)
+            w2 = bench.device_master(S["H"], S["I"], gen, device)
+            if e in hot:
+                layer.set_expert(e, B.BF16, w13, None, w2, None)
+            else:
+                q13, s13 = B.moe_quantize_weights(w13, B.INT4)
+                q2, s2 = B.moe_quantize_weights(w2, B.INT4)
+                layer.set_expert(e, B.INT4, q13, s13, q2, s2)
+        lg, x = synth.stack_logits(0, 0), synth.stack_x(0, 0)
+        dev_batches = [(torch.from_numpy(lg).to(device),
+                        torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device))]
+    elif name.startswith("decode"):
         base = synth.CONFIGS["qwen3_30b_decode"]
         tiers = {"decode": base.tiers, "decode-int4": [(base.E, synth.INT4)],
                  "decode-bf16": [(base.E, synth.BF16)]}[name]
@@ -121,21 +142,25 @@ def build_workload(name, device):
     bufs = layer.alloc_buffers(T, device)
     for _ in range(3):
         layer.forward(*dev_batches[0], bufs=bufs)
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        st = B.moe_get_device_status()
+        print(f"warm-up forward: status {st:#x}", flush=True)
     return layer, bufs
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "decode-int4", "decode-bf16", "mixtral-T1", "mixtral-T32"])
+                    choices=["decode", "decode-int4", "decode-bf16", "mixtral-T1", "mixtral-T32",
+                             "stack"])
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--sm-ghz", type=float, default=1.965, help="SM clock for cycle sums")
     ap.add_argument("--ctas", type=int, default=2, help="CTAs whose unit timeline is printed")
     ap.add_argument("--out", default=None)
     args = ap.parse_args()
     from mixed_precision_moe_b200 import build
-    os.environ["MOE_LIB_PATH"] = build.build(trace=True)
+    if not os.environ.get("MOE_LIB_PATH"):   # else: a profiling build given by the caller
+        os.environ["MOE_LIB_PATH"] = build.build(trace=True)
     import torch
     from mixed_precision_moe_b200 import binding as B
 
@@ -144,29 +169,53 @@ def main():
     L = B.lib()
     L.moe_ffn_trace_bytes.restype = C.c_size_t
     L.moe_ffn_trace_read.argtypes = [C.c_void_p, C.c_size_t]
+    L.moe_ffn_giveup_read.argtypes = [C.c_void_p, C.c_size_t]
+    giveup = np.zeros((CTAS, 4), np.int32)
+    assert L.moe_ffn_giveup_read(giveup.ctypes.data, giveup.nbytes) == 0   # clears it
     nbytes = int(L.moe_ffn_trace_bytes())
     assert nbytes == CTAS * UNITS * len(FIELDS) * 8, (nbytes, "trace layout changed")
     off, _, _, xp = bufs["permute"]
     y, ws = bufs["ffn"]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    launches, times = [], []
+    stream = torch.cuda.Stream(dev)
+    graph = torch.cuda.CUDAGraph()   # timed as the benchmark times it: a graph replay
+    with torch.cuda.graph(graph, stream=stream):
+        B.moe_grouped_ffn_mixed(layer, xp, off, y, ws, stream=stream)
+    torch.cuda.synchronize()
+    launches, times, kstamps = [], [], []
+    L.moe_ffn_kstamp_read.argtypes = [C.c_void_p, C.c_size_t]
     for _ in range(args.reps):
-        flush.zero_()
         torch.cuda.synchronize()
         assert L.moe_ffn_trace_reset() == 0
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        B.moe_grouped_ffn_mixed(layer, xp, off, y, ws)
-        e1.record()
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1) * 1e3)
         buf = np.zeros(nbytes // 8, np.int64)
         assert L.moe_ffn_trace_read(buf.ctypes.data, nbytes) == 0
         launches.append(buf.reshape(CTAS, UNITS, len(FIELDS)))
-    status = B.moe_get_device_status()
-    if status:
-        raise RuntimeError(f"device status {status:#x}")
-    res = {"workload": args.workload, "event_us": times,
+        ks = np.zeros((CTAS, 5), np.int64)
+        assert L.moe_ffn_kstamp_read(ks.ctypes.data, ks.nbytes) == 0
+        ks = ks[:148] if ks[148:].max() == 0 else ks
+        t0 = ks[:, 0].min()
+        rel = (ks - t0) / 1e3
+        kstamps.append({"entry_max": float(rel[:, 0].max()), "setup_done_mean": float(rel[:, 1].mean()),
+                        "table_done_mean": float(rel[:, 2].mean()), "table_done_max": float(rel[:, 2].max()),
+                        "final_barrier_min": float(rel[:, 3].min()),
+                        "final_barrier_mean": float(rel[:, 3].mean()),
+                        "exit_max": float(rel[:, 4].max())})
+        status = B.moe_get_device_status()
+        assert L.moe_ffn_giveup_read(giveup.ctypes.data, giveup.nbytes) == 0
+        gave = [(c, *giveup[c][:3].tolist()) for c in range(CTAS) if giveup[c][0]]
+        print(f"launch {len(times)}: {times[-1]:.1f} us, status {status:#x}, "
+              f"{len(gave)} CTAs gave up (cta, role, unit seq, thread): {gave[:12]}", flush=True)
+        if status:
+            raise RuntimeError(f"device status {status:#x}")
+    res = {"workload": args.workload, "event_us": times, "kernel_stamps_us": kstamps,
            "summary": summarise(launches[-1], args.sm_ghz)}
     rec = launches[-1]
     t0 = int(rec[rec[:, :, F["sched"]] != 0][:, F["sched"]].min())

@@ -117,6 +117,8 @@ def test_layer_stack_with_precision_swaps():
                 out = L.forward(torch.from_numpy(logits).to(dev), to_gpu_bf16(x), bufs=bufs,
                                 stream=compute)
             compute.synchronize()
+            status = B.moe_get_device_status()
+            assert status == 0, f"layer {layer} step {step}: device status {status:#x}"
             idx = bufs["route"][0].cpu().numpy()
             counts += np.bincount(idx.ravel(), minlength=E)
             if step not in sampled:
