@@ -174,7 +174,7 @@ int moe_grouped_ffn_mixed(moe_layer_t layer, const void* x_perm,
  * that loads the library until the process exits) and allocates nothing.
  *   Same arguments and results as moe_grouped_ffn_mixed, minus the workspace.
  *   Limit: moe_ffn_workspace_bytes(rows) must not exceed the scratch size, i.e.
- *   rows * I * 2 + 4096 <= 8 MiB; larger calls fail with MOE_ERR_UNSUPPORTED.
+ *   rows * I * 2 + 8192 <= 8 MiB; larger calls fail with MOE_ERR_UNSUPPORTED.
  *   The first call on a device looks up the scratch's device address (a
  *   cudaGetSymbolAddress with that device current); make that first call
  *   before any stream capture.  The address is cached per device index for
@@ -234,6 +234,56 @@ int moe_layer_forward(moe_layer_t layer, const float* logits, const void* x, int
  *   scales device fp16 [K/128][rows] */
 int moe_quantize_weights(const void* w_bf16, int rows, int K, moe_precision_t precision,
                          void* q_out, void* scales, void* stream);
+
+/* ---- Device-side precision management (DynaExq, arXiv 2511.15015, abstract:
+ * expert hotness estimated from router traces, a budget-feasible per-layer hot
+ * set, asynchronous promotion and demotion by swapping stable expert handles
+ * to fully materialised versions).  The counts, the selection and the handle
+ * swap all run on the device, stream-ordered, so no host synchronisation is
+ * needed between routing a batch and promoting its hot experts; only the
+ * host->device copies of newly promoted experts' BF16 weights are issued by
+ * the host (into slots registered below), from any stream. */
+
+/* Register (or, with NULL, unregister) a hotness counter: device uint32 [E].
+ * Every later moe_layer_forward of the layer adds, for each expert, the number
+ * of (token, slot) pairs routed to it in that forward (integer atomics: the
+ * totals do not depend on timing).  The caller owns and zeroes the buffer
+ * (moe_select_hot_experts can clear it). */
+int moe_layer_set_hotness_counter(moe_layer_t layer, unsigned int* counts);
+
+/* Size of the hot set that a memory budget allows: *n_hot = min(E,
+ * budget_bytes / (bytes of a BF16 expert - bytes of the same expert at
+ * `low`)), the bytes being the stored weights plus fp16 group-128 scales of
+ * the storage format above (ExactMoE Section 3.2 memory formula).  `low` is
+ * MOE_INT8 or MOE_INT4, the precision the cold experts stay at. */
+int moe_hot_set_size(moe_layer_t layer, size_t budget_bytes, moe_precision_t low, int* n_hot);
+
+/* Hot-set selection on the device: the n_hot experts with the highest counts,
+ * ties to the lower expert id, written to hot_ids (device int32 [n_hot]) in
+ * ascending id order.  counts: device uint32 [E], E <= 512; zero_counts != 0
+ * clears them afterwards (a new counting window starts).  Stream-ordered. */
+int moe_select_hot_experts(unsigned int* counts, int E, int n_hot, int zero_counts,
+                           int32_t* hot_ids, void* stream);
+
+/* Register the BF16 promotion slots: n_slots device buffers, each one
+ * expert's BF16 weights in the storage format above (slots[i].w13 bf16
+ * [2I][H], slots[i].w2 bf16 [H][I]; scales ignored), host array of n_slots.
+ * The library encodes one descriptor per slot; the caller keeps the buffers
+ * alive.  Synchronising (waits for the device, since forwards may read the
+ * slots it replaces); re-registering invalidates every promotion made from
+ * the old slots: apply a hot set again afterwards. */
+int moe_layer_set_bf16_slots(moe_layer_t layer, int n_slots, const moe_expert_weights* slots);
+
+/* Stream-ordered handle swap to a hot set: expert hot_ids[i] (device int32
+ * [n_hot], ascending, distinct, < E) now uses BF16 slot slot_base + i, and
+ * every other expert its base version (the one last installed by
+ * moe_set_expert_precision, which also replaces the expert's current handle).
+ * The slots' weights must be complete before the swap runs (record an event
+ * after their copies and make `stream` wait on it); forwards enqueued earlier
+ * keep the previous handles.  Fails with MOE_ERR_NOT_MATERIALIZED if an expert
+ * has no base version, MOE_ERR_INVALID_ARG if the slots are not registered. */
+int moe_apply_hot_set(moe_layer_t layer, const int32_t* hot_ids, int n_hot, int slot_base,
+                      void* stream);
 
 /* Read and clear the current device's status word (MOE_STATUS_* bits).
  * Synchronising. */

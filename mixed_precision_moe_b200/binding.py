@@ -41,6 +41,11 @@ SIGNATURES = {
     "moe_layer_forward": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _P]),
     "moe_quantize_weights": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "moe_get_device_status": (_I, [C.POINTER(C.c_uint)]),
+    "moe_layer_set_hotness_counter": (_I, [_P, _P]),
+    "moe_hot_set_size": (_I, [_P, _S, _I, C.POINTER(_I)]),
+    "moe_select_hot_experts": (_I, [_P, _I, _I, _I, _P, _P]),
+    "moe_layer_set_bf16_slots": (_I, [_P, _I, _P]),
+    "moe_apply_hot_set": (_I, [_P, _P, _I, _I, _P]),
 }
 
 
@@ -201,6 +206,16 @@ def moe_quantize_weights(w_bf16, precision, q_out=None, scales=None, stream=None
     return q_out, scales
 
 
+def moe_select_hot_experts(counts, n_hot, zero_counts=True, hot_ids=None, stream=None):
+    """counts: device uint32-as-int32 [E]; returns hot_ids (device int32 [n_hot])."""
+    _need(counts, torch.int32, "counts")
+    if hot_ids is None:
+        hot_ids = torch.empty(n_hot, dtype=torch.int32, device=counts.device)
+    _check(lib().moe_select_hot_experts(_ptr(counts), counts.numel(), n_hot, int(bool(zero_counts)),
+                                        _ptr(hot_ids), _stream(stream)))
+    return hot_ids
+
+
 def moe_get_device_status() -> int:
     v = C.c_uint(0)
     _check(lib().moe_get_device_status(C.byref(v)))
@@ -235,6 +250,35 @@ class MoELayer:
             ev.record(stream if stream is not None else torch.cuda.current_stream())
             self._retired.append((ev, old))
         self._retired = [(ev, t) for ev, t in self._retired if not ev.query()]
+
+    def set_hotness_counter(self, counts):
+        """counts: device int32 [E] (read as uint32) or None; later forwards add
+        their per-expert selection counts to it."""
+        if counts is not None:
+            _need(counts, torch.int32, "counts")
+            assert counts.numel() == self.E
+        self._hot = counts
+        _check(lib().moe_layer_set_hotness_counter(self.handle, _ptr(counts)))
+
+    def hot_set_size(self, budget_bytes, low=INT4) -> int:
+        n = C.c_int(0)
+        _check(lib().moe_hot_set_size(self.handle, int(budget_bytes), low, C.byref(n)))
+        return n.value
+
+    def set_bf16_slots(self, slots):
+        """slots: list of (w13 bf16 [2I, H], w2 bf16 [H, I]) device tensors."""
+        arr = (_ExpertWeights * max(1, len(slots)))()
+        for i, (w13, w2) in enumerate(slots):
+            _need(w13, torch.bfloat16, "slot w13")
+            _need(w2, torch.bfloat16, "slot w2")
+            arr[i] = _ExpertWeights(w13.data_ptr(), None, w2.data_ptr(), None)
+        self._slots = list(slots)
+        _check(lib().moe_layer_set_bf16_slots(self.handle, len(slots), arr))
+
+    def apply_hot_set(self, hot_ids, n_hot, slot_base, stream=None):
+        _need(hot_ids, torch.int32, "hot_ids")
+        _check(lib().moe_apply_hot_set(self.handle, _ptr(hot_ids), n_hot, slot_base,
+                                       _stream(stream)))
 
     def precision(self, e) -> int:
         p = C.c_int(0)

@@ -100,8 +100,9 @@ static_assert(sizeof(ExpertDesc) == 832, "descriptor layout");
 struct Unit {
   int e, prec, wrow0, nbox;  // expert, precision, first weight row (of each half), 128-row boxes
   int row0, nrows;           // rows of the token tile
-  int flags;                 // kUnitValid | kUnitGateUp
-  int need;                  // down unit: gate/up epilogue arrivals to wait for
+  int flags;                 // kUnitValid | kUnitGateUp | kUnitFma
+  int need;                  // gate/up arrivals of the expert (a down unit waits for them)
+  int ent;                   // the expert's entry in the unit table
 };
 constexpr int kUnitValid = 1, kUnitGateUp = 2, kUnitFma = 4;
 
@@ -118,8 +119,11 @@ struct Params {
   const int32_t* offsets;  // [E+1]
   __nv_bfloat16* h;        // [rows][I]: gate/up output, down input
   __nv_bfloat16* y;        // [rows][H]: down output
-  int* counter;            // work counter, zero at launch (unit = gridDim.x + count)
+  int* counter;            // [0] gate/up (swap) or unit (tile) counter, [1] down units
+                           // taken (swap), [2] ready slots reserved; zero at launch
   int* done;               // [E] finished gate/up epilogue warps per expert, zero at launch
+  int* ready;              // [E] swap mode: entry + 1 of each expert whose gate/up rows are
+                           // all published, in that order; zero at launch
   int rows;                // row capacity of x_perm, h and y_perm
   int E, H, I;
   int nwb_gu, nwb_dn;      // weight blocks per expert of each projection
@@ -329,10 +333,10 @@ __device__ __forceinline__ int tiles_of(int n, const Params& p) {
 // array: the experts with rows, with their first unit index; unit indices =
 // every gate/up unit, then every down unit, experts in the same order:
 //   swap kernel (decode): ascending id, so precisions are interleaved (hot
-//     experts sit at arbitrary ids) and the dynamic scheduler keeps
-//     latency-bound INT4 units and HBM-bound BF16 units running side by side
-//     on different SMs (measured 2.5 % faster on the mixed decode batch than
-//     INT4 first);
+//     experts sit at arbitrary ids) and HBM-bound BF16 units run beside the
+//     compute-bound CUDA-core units on other SMs (measured faster than putting
+//     either kind first); the scheduler hands out gate/up units in this order
+//     and down units in the order the experts become ready;
 //   tile kernel (prefill): INT4, then INT8, then BF16 experts (ascending id
 //     inside a class): the dequant-bound quantised units first, an LPT
 //     approximation that leaves the tail to the shorter BF16 units (measured
@@ -457,6 +461,7 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
   // gate/up arrivals: the 4 epilogue warps of a tensor-core unit, or every
   // dequant warp of a CUDA-core unit (an expert's units are all of one kind)
   un.need = (fma ? kDequantWarps : 4) * tiles_of(en.nrows, p) * p.nwb_gu;
+  un.ent = lo;
   return un;
 }
 
@@ -519,6 +524,17 @@ __device__ __forceinline__ void red_release_add(int* ptr, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ int atom_release_add(int* ptr, int v) {
+  int old;
+  asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v)
+               : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void st_release(int* ptr, int v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -555,6 +571,10 @@ __device__ void scheduler(const Params& p, const Smem& s) {
   int tseq = 0;
   (void)tseq;
   bool ok = true;
+  const int total_gu = *s.n_units_gu, total_dn = total - total_gu;
+  bool gu_left = true;
+  int dn_j = -1, scan_slot = 0, scan_cum = 0;  // swap mode: claimed down unit, ready-list cursor
+  const bool uniform_dn = total_dn == *s.n_entries * p.nwb_dn;  // every expert one token tile
   for (bool first = true;; first = false) {
     if (!first) {
       if (!mbar_wait(s.go, gph, abort_flag)) {
@@ -563,9 +583,73 @@ __device__ void scheduler(const Params& p, const Smem& s) {
       }
       gph ^= 1u;
     }
-    // the first unit of CTA b is unit b; later ones come from the counter
-    const int u = first ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.counter, 1);
-    Unit un = Unit{0, 0, 0, 0, 0, 0, 0, 0};
+    int u;
+    if (!kSwap) {
+      // tile mode: every gate/up unit, then every down unit, in order; the first
+      // unit of CTA b is unit b, later ones come from the counter
+      u = first ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.counter, 1);
+    } else if (first && (int)blockIdx.x < total_gu) {
+      u = blockIdx.x;
+    } else {
+      // swap mode: the next gate/up unit (the long units, on the critical
+      // path, go first); once none is left, a down unit of an expert whose
+      // gate/up rows are all published (experts in the order they became
+      // ready), waiting only if no expert is ready.  No SM waits on one expert
+      // while another expert's down units are ready.
+      // Down unit j (counted in the order the experts became ready) is taken by
+      // one atomicAdd, so takers never retry; its expert is found by walking
+      // the ready list from this scheduler's cursor (slot, down units before
+      // it), waiting only while that slot is not yet filled -- every later
+      // slot fills later, so no other down unit could be ready meanwhile.
+      u = -1;
+      const long long t0 = clock64();
+      while (u < 0) {
+        if (gu_left) {
+          const int g = (int)gridDim.x + atomicAdd(p.counter, 1);
+          if (g < total_gu) {
+            u = g;
+            break;
+          }
+          gu_left = false;
+        }
+        if (dn_j < 0) dn_j = atomicAdd(p.counter + 1, 1);
+        if (dn_j >= total_dn) {  // every down unit is taken: no work left
+          u = total;
+          break;
+        }
+        if (uniform_dn) {  // one token tile per expert: slot = j / (down units per expert)
+          const int v = ld_acquire(p.ready + dn_j / p.nwb_dn);
+          if (v != 0) {
+            u = s.ub_dn[v - 1] + dn_j % p.nwb_dn;
+            dn_j = -1;
+            break;
+          }
+          if (*abort_flag || clock64() - t0 > kWaitLimitCycles) break;
+          __nanosleep(200);
+          continue;
+        }
+        const int v = ld_acquire(p.ready + scan_slot);
+        if (v != 0) {
+          const int ent = v - 1;
+          const int nd = p.nwb_dn * tiles_of(s.entries[ent].nrows, p);
+          if (dn_j < scan_cum + nd) {
+            u = s.ub_dn[ent] + (dn_j - scan_cum);
+            dn_j = -1;
+            break;
+          }
+          scan_cum += nd;
+          ++scan_slot;
+          continue;
+        }
+        if (*abort_flag || clock64() - t0 > kWaitLimitCycles) break;
+        __nanosleep(200);
+      }
+      if (u < 0) {
+        ok = false;
+        break;
+      }
+    }
+    Unit un = Unit{0, 0, 0, 0, 0, 0, 0, 0, 0};
     if (u < total) {
       un = decode_unit<kSwap>(p, s, u);
       const ExpertDesc* d = p.descs + un.e;
@@ -937,15 +1021,21 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f +
 // Gate/up results: once this warp's h stores are done, publish them to the
 // down units of the expert (release counter; the proxy fence orders the
 // generic-proxy stores before any TMA read that the counter enables).
-__device__ __forceinline__ void publish_expert(const Params& p, int e, int lane) {
-  fence_proxy_async_global();
-  __threadfence();
-  __syncwarp();
-  if (lane == 0) red_release_add(p.done + e, 1);
-}
-
+// Ordering: each lane's proxy fence orders its generic-proxy h stores for the
+// async proxy (the TMA reads of the down units); __syncwarp orders the lanes'
+// stores before lane 0's release add, whose gpu-scope release covers them
+// (cumulativity), so no full fence is needed.  The arrival that completes the
+// expert's count appends the expert's entry to the ready list (swap mode's
+// scheduler takes down units from it): its atomic add reads every earlier
+// release on the counter, and the release store of the list entry carries
+// them on to the scheduler's acquire.
 __device__ __forceinline__ void publish_rows(const Params& p, const Unit& un, int lane) {
-  publish_expert(p, un.e, lane);
+  fence_proxy_async_global();
+  __syncwarp();
+  if (lane == 0) {
+    const int old = atom_release_add(p.done + un.e, 1);
+    if (old + 1 == un.need) st_release(p.ready + atomicAdd(p.counter + 2, 1), un.ent + 1);
+  }
 }
 
 // ------------------------------------------------------- CUDA-core units --
@@ -999,7 +1089,7 @@ __device__ __forceinline__ uint32_t nib_f32(uint32_t a, uint32_t b) {
 template <int N, bool kInt4>
 __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const Unit& un, int ft,
                                          uint32_t& st, uint32_t& sph, uint32_t& ffph,
-                                         uint32_t& fdph, int& pub_e, long long* tr) {
+                                         uint32_t& fdph, Unit& pub, long long* tr) {
   long long& tr_wait = tr[0];
   long long& tr_conv = tr[1];
   long long& tr_sync = tr[2];
@@ -1112,9 +1202,9 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
     advance(st, sph, ns);
     // the previous gate/up unit's h rows, stored a stage ago: publishing them
     // now costs little (the fence no longer waits for stores in flight)
-    if (pub_e >= 0) {
-      publish_expert(p, pub_e, lane);
-      pub_e = -1;
+    if (pub.flags & kUnitValid) {
+      publish_rows(p, pub, lane);
+      pub.flags = 0;
     }
   }
   const long long c3 = FFN_CLOCK();
@@ -1138,7 +1228,7 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
         if (c == n && n < un.nrows)
           p.h[(size_t)(un.row0 + n) * p.I + un.wrow0 + 16 * j + rsub] =
               __float2bfloat16_rn(silu_mul(acc[j][n], acc[j + 4][n]));
-    pub_e = un.e;  // published by the caller later (deferred publication)
+    pub = un;  // published later (deferred publication)
   } else {
 #pragma unroll
     for (int j = 0; j < 8; ++j)
@@ -1154,16 +1244,16 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
 
 template <bool kInt4>
 __device__ bool fma_dispatch(const Params& p, const Smem& s, const Unit& un, int ft, uint32_t& st,
-                             uint32_t& sph, uint32_t& ffph, uint32_t& fdph, int& pub_e,
+                             uint32_t& sph, uint32_t& ffph, uint32_t& fdph, Unit& pub,
                              long long* tr) {
   static_assert(kFmaRows >= 1 && kFmaRows <= 4, "CUDA-core tiles of 1 to 4 rows");
   if (kFmaRows >= 4 && un.nrows == 4)
-    return fma_unit<4, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+    return fma_unit<4, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
   if (kFmaRows >= 3 && un.nrows == 3)
-    return fma_unit<3, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+    return fma_unit<3, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
   if (kFmaRows >= 2 && un.nrows == 2)
-    return fma_unit<2, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
-  return fma_unit<1, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+    return fma_unit<2, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+  return fma_unit<1, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
 }
 
 // One staging slot holds an INT4 group (128 K-elements = two k-blocks) or an
@@ -1197,16 +1287,16 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
   // stage into the next CUDA-core unit, when their stores have landed -- and
   // always before this warp could block on anything a down unit's wait could
   // hold up: the unit ring, or an INT8/INT4 tensor-core unit.
-  int pub_e = -1;
+  Unit pub = Unit{0, 0, 0, 0, 0, 0, 0, 0, 0};  // flags != 0: a publication is pending
   bool ok = true;
   int tseq = -1;
   const bool tracer = warp == 2 && lane == 0;
   (void)tseq;
   (void)tracer;
   for (;;) {
-    if (pub_e >= 0 && !mbar_try_wait(&s.ufull[us], uph)) {
-      publish_expert(p, pub_e, lane);
-      pub_e = -1;
+    if ((pub.flags & kUnitValid) && !mbar_try_wait(&s.ufull[us], uph)) {
+      publish_rows(p, pub, lane);
+      pub.flags = 0;
     }
     if (!mbar_wait(&s.ufull[us], uph, abort_flag)) {
       ok = false;
@@ -1219,9 +1309,9 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
     if (!(un.flags & kUnitValid)) break;
     ++tseq;
     const int nkb = unit_nkb(p, un);
-    if (pub_e >= 0 && !unit_fma(un)) {
-      publish_expert(p, pub_e, lane);
-      pub_e = -1;
+    if ((pub.flags & kUnitValid) && !unit_fma(un)) {
+      publish_rows(p, pub, lane);
+      pub.flags = 0;
     }
     if (un.prec == MOE_BF16) {
       for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
@@ -1231,8 +1321,8 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
     if (unit_fma(un)) {
       long long tr[5] = {0, 0, 0, 0, 0};
       ok = un.prec == MOE_INT4
-               ? fma_dispatch<true>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr)
-               : fma_dispatch<false>(p, s, un, ft, st, sph, ffph, fdph, pub_e, tr);
+               ? fma_dispatch<true>(p, s, un, ft, st, sph, ffph, fdph, pub, tr)
+               : fma_dispatch<false>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
       if (!ok) break;
       if (tracer) {
         FFN_TRACE_SET(tseq, kTrDqEnd, FFN_TRACE_NS());
@@ -1319,7 +1409,7 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
       FFN_TRACE_SET(tseq, kTrDqStore, tr_store);
     }
   }
-  if (pub_e >= 0) publish_expert(p, pub_e, lane);
+  if (pub.flags & kUnitValid) publish_rows(p, pub, lane);
   if (!ok) give_up(s, 5, tseq);
 }
 
@@ -1546,6 +1636,7 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.accempty[ebuf]);
     const long long cp = FFN_CLOCK();
+    (void)cp;
     if (gu) publish_rows(p, un, lane);
     if (tracer) {
       FFN_TRACE_SET(tseq, kTrEpiEnd, FFN_TRACE_NS());
@@ -1643,14 +1734,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   FFN_KSTAMP(4);
 }
 
+// Stream-ordered swap of a layer's whole descriptor table to a hot set (the
+// DynaExq abstract's asynchronous promotion through stable expert handles):
+// expert e gets the descriptor of BF16 slot slot_base + i if e == hot_ids[i]
+// (hot_ids ascending, n entries), else its base version (the one installed by
+// moe_set_expert_precision).  One CTA per expert.  The weights behind every
+// descriptor must be complete before this kernel runs (stream order).
+__global__ void apply_hot_set_kernel(ExpertDesc* __restrict__ descs, int* __restrict__ prec,
+                                     const ExpertDesc* __restrict__ base,
+                                     const ExpertDesc* __restrict__ slots,
+                                     const int32_t* __restrict__ hot_ids, int n, int slot_base) {
+  const int e = blockIdx.x;
+  int lo = 0, hi = n;  // first index with hot_ids[index] >= e
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (hot_ids[mid] < e)
+      lo = mid + 1;
+    else
+      hi = mid;
+  }
+  const bool hot = lo < n && hot_ids[lo] == e;
+  const ExpertDesc* src = hot ? slots + slot_base + lo : base + e;
+  for (int v = threadIdx.x; v < (int)(sizeof(ExpertDesc) / 16); v += blockDim.x)
+    reinterpret_cast<uint4*>(descs + e)[v] = reinterpret_cast<const uint4*>(src)[v];
+  if (threadIdx.x == 0) prec[e] = src->prec;
+  tmap_release();
+}
+
 // Stream-ordered install of one expert descriptor (a by-value kernel argument,
 // so the host buffer needs no lifetime beyond the launch) and of its precision
 // in the compact precision array.
-__global__ void write_desc_kernel(ExpertDesc* dst, int* prec_dst,
+// dst2 (optional): a second copy (the layer's base table).
+__global__ void write_desc_kernel(ExpertDesc* dst, int* prec_dst, ExpertDesc* dst2,
                                   const __grid_constant__ ExpertDesc d) {
   const int i = threadIdx.x;
-  for (int v = i; v < (int)(sizeof(ExpertDesc) / 16); v += blockDim.x)
+  for (int v = i; v < (int)(sizeof(ExpertDesc) / 16); v += blockDim.x) {
     reinterpret_cast<uint4*>(dst)[v] = reinterpret_cast<const uint4*>(&d)[v];
+    if (dst2 != nullptr) reinterpret_cast<uint4*>(dst2)[v] = reinterpret_cast<const uint4*>(&d)[v];
+  }
   if (i == 0) *prec_dst = d.prec;
   tmap_release();
 }

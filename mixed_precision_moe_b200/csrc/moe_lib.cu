@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -165,10 +166,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Scheduler counters at the end of the FFN workspace: the work counter, then
-// (from int 16) one gate/up completion counter per expert.
-constexpr size_t kFfnCounterBytes = 4096;
-size_t ffn_counter_bytes(int E) { return (16 + (size_t)E) * sizeof(int); }
+// Scheduler counters at the end of the FFN workspace: the work counters, then
+// (from int 16) one gate/up completion counter per expert and the ready list
+// of experts ([E]).
+constexpr size_t kFfnCounterBytes = 8192;
+size_t ffn_counter_bytes(int E) { return (16 + 2 * (size_t)E) * sizeof(int); }
+static_assert((16 + 2 * 512) * sizeof(int) <= kFfnCounterBytes, "counter space");
 
 int num_sms(int device) {
   int n = 0;
@@ -181,9 +184,13 @@ int num_sms(int device) {
 struct moe_layer {
   int H, I, E, k;
   int device;
-  moe::ffn::ExpertDesc* d_descs;  // [E], device
+  moe::ffn::ExpertDesc* d_descs;  // [E], device: the table the forwards read
   int* d_prec;                    // [E], device: compact copy of the precisions
-  std::vector<int> prec;          // host shadow, -1 = unset
+  moe::ffn::ExpertDesc* d_base;   // [E], device: the versions installed by set_expert_precision
+  moe::ffn::ExpertDesc* d_slots = nullptr;  // [n_slots], device: BF16 promotion slots
+  int n_slots = 0;
+  unsigned int* hot = nullptr;    // device [E]: selection counts (NULL: not counted)
+  std::vector<int> prec;          // host shadow of the base versions, -1 = unset
 };
 
 extern "C" {
@@ -238,17 +245,19 @@ int moe_layer_create(int H, int I, int E, int k, moe_layer_t* out) {
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   moe::ffn::ExpertDesc* d = nullptr;
   const size_t table = sizeof(moe::ffn::ExpertDesc) * E;
-  MOE_CUDA_TRY(cudaMalloc(&d, table + sizeof(int) * E));
-  int* dp = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(d) + table);
-  // All bytes 0xFF: prec = -1 (unset) for every expert, in both arrays.
-  cudaError_t e1 = cudaMemset(d, 0xFF, table + sizeof(int) * E);
+  // active table, then the base table, then the compact precisions
+  MOE_CUDA_TRY(cudaMalloc(&d, 2 * table + sizeof(int) * E));
+  int* dp = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(d) + 2 * table);
+  // All bytes 0xFF: prec = -1 (unset) for every expert, in every array.
+  cudaError_t e1 = cudaMemset(d, 0xFF, 2 * table + sizeof(int) * E);
   cudaError_t e2 = cudaDeviceSynchronize();
   if (e1 != cudaSuccess || e2 != cudaSuccess) {
     cudaFree(d);
     return fail(MOE_ERR_CUDA, "descriptor table init failed: %s",
                 cudaGetErrorString(e1 != cudaSuccess ? e1 : e2));
   }
-  moe_layer* L = new moe_layer{H, I, E, k, dev, d, dp, std::vector<int>(E, -1)};
+  moe_layer* L = new moe_layer{H, I, E, k, dev, d, dp, d + E};
+  L->prec.assign(E, -1);
   *out = L;
   return ok();
 }
@@ -257,6 +266,7 @@ int moe_layer_destroy(moe_layer_t layer) {
   MOE_CHECK(layer != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
   cudaDeviceSynchronize();
   cudaError_t e = cudaFree(layer->d_descs);
+  if (layer->d_slots != nullptr) cudaFree(layer->d_slots);
   delete layer;
   MOE_CHECK(e == cudaSuccess, MOE_ERR_CUDA, "cudaFree failed: %s", cudaGetErrorString(e));
   return ok();
@@ -287,7 +297,8 @@ int moe_set_expert_precision(moe_layer_t L, int expert, moe_precision_t precisio
   d.s2 = prec == MOE_BF16 ? nullptr : static_cast<const __half*>(w->s2);
   d.prec = prec;
   moe::ffn::write_desc_kernel<<<1, 32, 0, as_stream(stream)>>>(L->d_descs + expert,
-                                                               L->d_prec + expert, d);
+                                                               L->d_prec + expert,
+                                                               L->d_base + expert, d);
   MOE_CUDA_TRY(cudaGetLastError());
   L->prec[expert] = prec;
   return ok();
@@ -320,9 +331,12 @@ int moe_route_topk(const float* logits, int T, int E, int k, int renormalize, in
   return ok();
 }
 
-int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int H,
-                int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row, void* x_perm,
-                void* stream) {
+}  // extern "C"
+
+namespace {
+int permute_impl(const int32_t* topk_idx, const void* x, int T, int E, int k, int H,
+                 int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row, void* x_perm,
+                 unsigned int* hot, void* stream) {
   MOE_CHECK(T >= 0, MOE_ERR_INVALID_ARG, "T=%d < 0", T);
   MOE_CHECK(E >= 1 && E <= 512, MOE_ERR_UNSUPPORTED, "E=%d outside [1, 512]", E);
   MOE_CHECK(k >= 1 && k <= 16, MOE_ERR_INVALID_ARG, "k=%d outside [1, 16]", k);
@@ -350,7 +364,7 @@ int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int
   if (T <= 2 * moe::kPermuteChunk) {  // one CTA
     MOE_CUDA_TRY(launch_pdl(moe::permute_index_kernel, dim3(1), dim3(moe::kPermuteThreads), smem,
                             s, topk_idx, T, E, k, expert_offsets, perm_token, dest_row,
-                            static_cast<const int32_t*>(nullptr)));
+                            static_cast<const int32_t*>(nullptr), hot));
   } else {
     // Split over CTAs of kPermuteChunk tokens: per-CTA expert counts first.  They
     // are kept in x_perm (nblk * E ints <= T * k * H * 2 bytes), which the row
@@ -363,7 +377,7 @@ int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int
                             (size_t)E * sizeof(int32_t), s, topk_idx, T, E, k, counts));
     MOE_CUDA_TRY(launch_pdl(moe::permute_index_kernel, dim3(nblk), dim3(moe::kPermuteThreads),
                             smem, s, topk_idx, T, E, k, expert_offsets, perm_token, dest_row,
-                            static_cast<const int32_t*>(counts)));
+                            static_cast<const int32_t*>(counts), hot));
   }
   const int vec = H / 8;
   const long long nvec = (long long)T * k * vec;
@@ -373,6 +387,16 @@ int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int
                           static_cast<const uint4*>(x), perm_token, expert_offsets, E, vec,
                           static_cast<uint4*>(x_perm)));
   return ok();
+}
+}  // namespace
+
+extern "C" {
+
+int moe_permute(const int32_t* topk_idx, const void* x, int T, int E, int k, int H,
+                int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row, void* x_perm,
+                void* stream) {
+  return permute_impl(topk_idx, x, T, E, k, H, expert_offsets, perm_token, dest_row, x_perm,
+                      nullptr, stream);
 }
 
 int moe_ffn_workspace_bytes(moe_layer_t L, int rows, size_t* bytes) {
@@ -468,7 +492,7 @@ int route_permute_gather_small(moe_layer_t L, const float* logits, const void* x
                           logits, static_cast<const uint4*>(x), T, E, k, renormalize, H / 8,
                           topk_idx, topk_w, expert_offsets, perm_token, dest_row,
                           static_cast<uint4*>(x_perm), counters,
-                          (int)(ffn_counter_bytes(E) / sizeof(int))));
+                          (int)(ffn_counter_bytes(E) / sizeof(int)), L->hot));
   return ok();
 }
 
@@ -537,7 +561,7 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
   }
 
   Params prm{L->d_descs, L->d_prec, expert_offsets, h, static_cast<__nv_bfloat16*>(y_perm),
-             counters, counters + 16, rows, L->E, L->H, L->I,
+             counters, counters + 16, counters + 16 + L->E, rows, L->E, L->H, L->I,
              swap ? L->I / 64 : L->I / 128, swap ? L->H / 128 : (L->H + 255) / 256,
              xbox, xrows, ns, nq, acc_stride, a_col, fma_rows};
 
@@ -671,8 +695,8 @@ int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, 
                                  ffn_counter_bytes(L->E), as_stream(stream)));
     rc = moe_route_topk(logits, T, L->E, L->k, renormalize, topk_idx, topk_w, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_permute(topk_idx, x, T, L->E, L->k, L->H, expert_offsets, perm_token, dest_row,
-                     x_perm, stream);
+    rc = permute_impl(topk_idx, x, T, L->E, L->k, L->H, expert_offsets, perm_token, dest_row,
+                      x_perm, L->hot, stream);
     if (rc != MOE_OK) return rc;
   }
   rc = grouped_ffn_impl(L, x_perm, expert_offsets, T * L->k, y_perm, workspace, workspace_bytes,
@@ -698,6 +722,79 @@ int moe_quantize_weights(const void* w_bf16, int rows, int K, moe_precision_t pr
   moe::quantize_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(
       static_cast<const uint16_t*>(w_bf16), rows, K, prec, static_cast<uint8_t*>(q_out),
       static_cast<uint16_t*>(scales));
+  MOE_CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+int moe_layer_set_hotness_counter(moe_layer_t L, unsigned int* counts) {
+  MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  MOE_CHECK(counts == nullptr || aligned(counts, 4), MOE_ERR_UNSUPPORTED, "misaligned counts");
+  L->hot = counts;
+  return ok();
+}
+
+int moe_hot_set_size(moe_layer_t L, size_t budget_bytes, moe_precision_t low, int* n_hot) {
+  MOE_CHECK(L != nullptr && n_hot != nullptr, MOE_ERR_INVALID_ARG, "null argument");
+  MOE_CHECK(low == MOE_INT8 || low == MOE_INT4, MOE_ERR_INVALID_ARG,
+            "the precision experts are promoted from must be INT8 or INT4");
+  const size_t P = (size_t)3 * L->H * L->I;
+  const size_t bf16 = 2 * P, q = (low == MOE_INT4 ? P / 2 : P) + P / 64;  // weights + fp16 scales
+  const size_t n = budget_bytes / (bf16 - q);
+  *n_hot = (int)std::min<size_t>(n, (size_t)L->E);
+  return ok();
+}
+
+int moe_select_hot_experts(unsigned int* counts, int E, int n_hot, int zero_counts,
+                           int32_t* hot_ids, void* stream) {
+  MOE_CHECK(E >= 1 && E <= moe::kSelectThreads, MOE_ERR_UNSUPPORTED, "E=%d outside [1, 512]", E);
+  MOE_CHECK(n_hot >= 0 && n_hot <= E, MOE_ERR_INVALID_ARG, "n_hot=%d outside [0, E]", n_hot);
+  MOE_CHECK(counts != nullptr && (hot_ids != nullptr || n_hot == 0), MOE_ERR_INVALID_ARG,
+            "null pointer");
+  MOE_CUDA_TRY(launch_pdl(moe::select_hot_kernel, dim3(1), dim3(moe::kSelectThreads), 0,
+                          as_stream(stream), counts, E, n_hot, zero_counts, hot_ids));
+  return ok();
+}
+
+int moe_layer_set_bf16_slots(moe_layer_t L, int n_slots, const moe_expert_weights* slots) {
+  MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  MOE_CHECK(n_slots >= 0 && n_slots <= 4 * L->E, MOE_ERR_INVALID_ARG, "n_slots=%d", n_slots);
+  MOE_CHECK(n_slots == 0 || slots != nullptr, MOE_ERR_INVALID_ARG, "null slots");
+  std::vector<moe::ffn::ExpertDesc> h((size_t)n_slots);
+  for (int i = 0; i < n_slots; ++i) {
+    MOE_CHECK(slots[i].w13 != nullptr && slots[i].w2 != nullptr, MOE_ERR_INVALID_ARG,
+              "null weight pointer in slot %d", i);
+    MOE_CHECK(aligned(slots[i].w13, 16) && aligned(slots[i].w2, 16), MOE_ERR_UNSUPPORTED,
+              "slot buffers must be 16-byte aligned");
+    memset(&h[i], 0, sizeof h[i]);
+    const int rc = encode_weights(&h[i], &slots[i], MOE_BF16, L->H, L->I);
+    if (rc != MOE_OK) return rc;
+    h[i].prec = MOE_BF16;
+  }
+  cudaDeviceSynchronize();  // no forward may still read the slots being replaced
+  if (L->d_slots != nullptr) cudaFree(L->d_slots);
+  L->d_slots = nullptr;
+  L->n_slots = 0;
+  if (n_slots > 0) {
+    MOE_CUDA_TRY(cudaMalloc(&L->d_slots, sizeof(moe::ffn::ExpertDesc) * n_slots));
+    MOE_CUDA_TRY(cudaMemcpy(L->d_slots, h.data(), sizeof(moe::ffn::ExpertDesc) * n_slots,
+                            cudaMemcpyHostToDevice));
+  }
+  L->n_slots = n_slots;
+  return ok();
+}
+
+int moe_apply_hot_set(moe_layer_t L, const int32_t* hot_ids, int n_hot, int slot_base,
+                      void* stream) {
+  MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
+  MOE_CHECK(n_hot >= 0 && n_hot <= L->E, MOE_ERR_INVALID_ARG, "n_hot=%d outside [0, E]", n_hot);
+  MOE_CHECK(slot_base >= 0 && slot_base + n_hot <= L->n_slots, MOE_ERR_INVALID_ARG,
+            "slots [%d, %d) outside the %d registered slots", slot_base, slot_base + n_hot,
+            L->n_slots);
+  MOE_CHECK(n_hot == 0 || hot_ids != nullptr, MOE_ERR_INVALID_ARG, "null hot_ids");
+  for (int e = 0; e < L->E; ++e)
+    MOE_CHECK(L->prec[e] >= 0, MOE_ERR_NOT_MATERIALIZED, "expert %d has no weights", e);
+  moe::ffn::apply_hot_set_kernel<<<L->E, 64, 0, as_stream(stream)>>>(
+      L->d_descs, L->d_prec, L->d_base, L->d_slots, hot_ids, n_hot, slot_base);
   MOE_CUDA_TRY(cudaGetLastError());
   return ok();
 }

@@ -175,7 +175,8 @@ __global__ void __launch_bounds__(kPermuteThreads, 1)
     permute_index_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
                          int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
                          int32_t* __restrict__ dest_row,
-                         const int32_t* __restrict__ blk_counts) {
+                         const int32_t* __restrict__ blk_counts,
+                         unsigned int* __restrict__ hot) {
   extern __shared__ int32_t psm[];
   int32_t* base = psm;                                          // [warps][E]
   uint32_t* mask = reinterpret_cast<uint32_t*>(psm + kPermuteWarps * E);  // [warps][E]
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(kPermuteThreads, 1)
         const int c = tot[e];
         tot[e] = run + (split ? pre[e] : 0);
         if (lead) offsets[e] = run;
+        if (lead && hot != nullptr && c != 0) atomicAdd(hot + e, (unsigned int)c);
         run += c;
       }
     }
@@ -351,7 +353,8 @@ __global__ void __launch_bounds__(kFrontThreads, 1)
                                 int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                                 int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
                                 int32_t* __restrict__ dest_row, uint4* __restrict__ x_perm,
-                                int* __restrict__ zero_ptr, int zero_n) {
+                                int* __restrict__ zero_ptr, int zero_n,
+                                unsigned int* __restrict__ hot) {
   extern __shared__ int32_t fsm[];
   const int pairs = T * k;
   int32_t* sidx = fsm;                                     // [pairs] expert of pair (t, j)
@@ -406,6 +409,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1)
         const int c = base[e];
         base[e] = run;
         if (lead) offsets[e] = run;
+        if (lead && hot != nullptr && c != 0) atomicAdd(hot + e, (unsigned int)c);
         run += c;
       }
     }
@@ -545,6 +549,42 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
                                        ((qv[3] + 8) << 12));
     *reinterpret_cast<uint16_t*>(q + (size_t)row * (K / 2) + g * 64 + lane * 2) = packed;
   }
+}
+
+// ----------------------------------------------------------- hot experts --
+// Hot set of one layer (DynaExq abstract: a per-layer set of hot experts,
+// estimated from router traces, under a memory budget): the n experts with the
+// highest selection counts, ties to the lower id, written in ascending id
+// order.  One CTA, one thread per expert (E <= 512): an expert's rank is the
+// number of experts before it in (count descending, id ascending) order, found
+// by comparing with every count; its output slot is the number of selected
+// experts with a lower id.  zero != 0 clears the counts afterwards (a new
+// counting window starts).
+constexpr int kSelectThreads = 512;
+
+__global__ void __launch_bounds__(kSelectThreads)
+    select_hot_kernel(unsigned int* __restrict__ counts, int E, int n, int zero,
+                      int32_t* __restrict__ hot_ids) {
+  __shared__ unsigned int c[kSelectThreads];
+  __shared__ int sel[kSelectThreads];
+  const int e = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  c[e] = e < E ? counts[e] : 0u;
+  __syncthreads();
+  int rank = 0;
+  if (e < E) {
+    const unsigned int mine = c[e];
+    for (int j = 0; j < E; ++j) rank += (c[j] > mine) || (c[j] == mine && j < e);
+  }
+  sel[e] = (e < E && rank < n) ? 1 : 0;
+  __syncthreads();
+  if (sel[e]) {
+    int pos = 0;
+    for (int j = 0; j < e; ++j) pos += sel[j];
+    hot_ids[pos] = e;
+  }
+  if (zero && e < E) counts[e] = 0u;
 }
 
 }  // namespace moe

@@ -59,7 +59,7 @@ def test_noalloc_refuses_calls_larger_than_its_scratch():
     H, I = 256, 512
     layer = B.MoELayer(H, I, 2, 2)
     try:
-        rows = (limit - 4096) // (2 * I) + 1          # one row past the limit
+        rows = (limit - 8192) // (2 * I) + 1          # one row past the limit
         xp = torch.zeros((rows, H), dtype=torch.bfloat16, device="cuda")
         off = torch.tensor([0, rows, rows], dtype=torch.int32, device="cuda")
         with pytest.raises(B.MoeError) as ei:
