@@ -285,7 +285,7 @@ def run_workload(cfg, steps, warmup, device, with_e2e, dist_barrier):
                 ev[i][1].record(stream)
             torch.cuda.synchronize()
         res["e2e_ms"] = float(np.mean([a.elapsed_time(b) for a, b in ev]))
-        for b in range(n_batches):   # same inputs, same deterministic kernels
+        for b in range(min(n_batches, max(warmup, steps))):   # the batches the loops ran
             if not torch.equal(outs[b].to(device), ref_out[b]):
                 raise RuntimeError(f"end-to-end output of batch {b} differs from the graph's")
         res["h2d_bytes"] = lg_bytes + cfg.T * cfg.H * 2   # the logits and x bytes of a step
@@ -356,7 +356,7 @@ def device_master(rows, K, gen, device, std=0.02):
     return (torch.randn((rows, K), generator=gen, device=device) * std).to(torch.bfloat16)
 
 
-def mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src):
+def mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src, batches=None):
     """Mixtral-8x7B-shaped layer, all experts INT4, uniform logits, over the
     token batch sweep: per batch the layer step, the grouped FFN alone and the
     FFN against its bound, max(expert bytes / HBM, flops / bf16 peak)."""
@@ -381,7 +381,8 @@ def mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src):
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     points = []
-    for T in synth.MIXTRAL_BATCHES:
+    batches = list(batches or synth.MIXTRAL_BATCHES)
+    for T in batches:
         cfg = synth.mixtral_config(T)
         n_b = 2
         dev_b = []
@@ -422,37 +423,39 @@ def mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src):
         raise RuntimeError(f"device status {status:#x} after the sweep")
     layer.close()
     return {"workload": f"mixtral_8x7b sweep: H={H} I={I} E={E} top-{k}, all experts INT4 "
-                        f"group-128, uniform N(0,1) logits, T in {list(synth.MIXTRAL_BATCHES)}",
+                        f"group-128, uniform N(0,1) logits, T in {batches}",
             "data": "synthetic (logits and x host-seeded; experts drawn on the device)",
             "timing": f"CUDA graphs, {steps} timed replays after {warmup}, L2 flushed between",
             "peaks": {"hbm_gbs": hbm_gbs, "bf16_tflops": tf_burst, "source": peak_src},
             "points": points, "clocks": clk}
 
 
-def _hot_set(counts, n):
-    """The n most selected experts, ties to the lower id (sorted ids)."""
-    order = np.lexsort((np.arange(len(counts)), -counts))
-    return np.sort(order[:n])
-
-
-def stack_run(args, device, hbm_gbs, peak_src):
-    """Qwen3-80B-scale stack: 4 layers (H 2048, I 512, 512 experts, top-10) at
-    decode batch 32 for 256 steps, Zipf(1.2) routing whose popularity order is
-    redrawn every 64 steps.  Every expert stays resident as INT4; the 64
-    experts of each layer selected most often in the previous 64 steps are
-    BF16.  At each step 64 m the promoted experts' bf16 masters are copied from
-    pinned host memory on a side stream, the compute stream waits on that copy,
-    and every change goes through moe_set_expert_precision before the step's
-    forward.  A step is the four layer forwards (one CUDA graph each)."""
+def stack_run(args, device, hbm_gbs, peak_src, n_layers=None, n_steps=None):
+    """Qwen3-80B-scale stack: layers of H 2048, I 512, 512 experts, top-10 at
+    decode batch 32, Zipf(1.2) routing whose popularity order is redrawn every
+    64 steps (4 layers x 256 steps by default).  Every expert stays resident as
+    INT4; the 64 hottest are BF16, managed on the device per layer
+    (mixed_precision_moe_b200.precision_manager): the routing kernels count the
+    selections, the hot set of the last 64-step window is selected on the device
+    at each step 64 m, the promoted experts' BF16 weights are copied into the
+    idle slot set on a side stream once the selection is known (a non-blocking
+    event query; experts already BF16 are copied device to device), and the
+    handle swap runs on the device once the copies are done.  The compute stream
+    never waits on a copy in flight; the gap between consecutive steps is the
+    stall an update costs.  The host runs at most 8 steps ahead of the GPU.  A step is every layer's forward (one CUDA graph per
+    layer and step)."""
     from mixed_precision_moe_b200 import binding as B
+    from mixed_precision_moe_b200.precision_manager import PrecisionManager
     S = synth.STACK
-    nl, H, I, E, k, T = S["layers"], S["H"], S["I"], S["E"], S["k"], S["T"]
-    steps, epoch, n_hot = S["steps"], S["epoch"], S["n_hot"]
+    nl = n_layers or S["layers"]
+    steps = n_steps or S["steps"]
+    H, I, E, k, T = S["H"], S["I"], S["E"], S["k"], S["T"]
+    epoch, n_hot = S["epoch"], S["n_hot"]
     compute = torch.cuda.Stream(device)
     copy = torch.cuda.Stream(device)
     gen = torch.Generator(device=device)
     gen.manual_seed(S["seed"])
-    layers, int4, host13, host2, bf16, hot, prec_hist = [], [], [], [], [], [], []
+    layers, mgrs, keep = [], [], []
     chunk = 64
     for l in range(nl):
         L = B.MoELayer(H, I, E, k)
@@ -468,108 +471,74 @@ def stack_run(args, device, hbm_gbs, peak_src):
                 q.append(B.moe_quantize_weights(w13[j], B.INT4) +
                          B.moe_quantize_weights(w2[j], B.INT4))
             del w13, w2
-        first = set(np.argsort(synth.stack_ranks(l, 0), kind="stable")[:n_hot].tolist())
-        mine = {}
         for e in range(E):
-            if e in first:
-                d13 = h13[e].to(device)
-                d2 = h2[e].to(device)
-                mine[e] = (d13, d2)
-                L.set_expert(e, B.BF16, d13, None, d2, None)
-            else:
-                q13, s13, q2, s2 = q[e]
-                L.set_expert(e, B.INT4, q13, s13, q2, s2)
+            q13, s13, q2, s2 = q[e]
+            L.set_expert(e, B.INT4, q13, s13, q2, s2, stream=compute)
+        assert L.hot_set_size(n_hot * (expert_bytes(synth.BF16, H, I) -
+                                       expert_bytes(synth.INT4, H, I))) == n_hot
+        mgr = PrecisionManager(L, [(h13[e], h2[e]) for e in range(E)], n_hot, device, copy)
+        mgr.bootstrap(np.argsort(synth.stack_ranks(l, 0), kind="stable")[:n_hot], compute)
         layers.append(L)
-        int4.append(q)
-        host13.append(h13)
-        host2.append(h2)
-        bf16.append(mine)
-        hot.append(np.array(sorted(first)))
+        mgrs.append(mgr)
+        keep.append((q, h13, h2))
     torch.cuda.synchronize()
-    prec_hist.append([np.isin(np.arange(E), hot[l]) for l in range(nl)])   # True = BF16
 
-    # every step's inputs on the device; routing of every step kept for the hot sets
     lg_all = torch.empty((steps, nl, T, E), dtype=torch.float32, device=device)
     x_all = torch.empty((steps, nl, T, H), dtype=torch.bfloat16, device=device)
-    for s in range(steps):
+    for st in range(steps):
         for l in range(nl):
-            lg_all[s, l].copy_(torch.from_numpy(synth.stack_logits(l, s)))
-            x_all[s, l].copy_(torch.from_numpy(synth.stack_x(l, s).view(np.int16))
-                              .view(torch.bfloat16))
+            lg_all[st, l].copy_(torch.from_numpy(synth.stack_logits(l, st)))
+            x_all[st, l].copy_(torch.from_numpy(synth.stack_x(l, st).view(np.int16))
+                               .view(torch.bfloat16))
     hist = torch.zeros((steps, nl, T, k), dtype=torch.int32, device=device)
     bufs = [layers[l].alloc_buffers(T, device) for l in range(nl)]
     with torch.cuda.stream(compute):
         for l in range(nl):
             layers[l].forward(lg_all[0, l], x_all[0, l], bufs=bufs[l], stream=compute)
     torch.cuda.synchronize()
+    for m in mgrs:   # the warm-up forwards counted: start the first window clean
+        m.counts.zero_()
     pool = torch.cuda.graph_pool_handle()
     graphs = []
     with torch.cuda.stream(compute):
-        for s in range(steps):
+        for st in range(steps):
             row = []
             for l in range(nl):
                 b = dict(bufs[l])
-                b["route"] = (hist[s, l], bufs[l]["route"][1])
+                b["route"] = (hist[st, l], bufs[l]["route"][1])
                 g = torch.cuda.CUDAGraph()
                 g.capture_begin(pool=pool)
-                layers[l].forward(lg_all[s, l], x_all[s, l], bufs=b, stream=compute)
+                layers[l].forward(lg_all[st, l], x_all[st, l], bufs=b, stream=compute)
                 g.capture_end()
                 row.append(g)
             graphs.append(row)
+    torch.cuda.synchronize()
+    for m in mgrs:   # capture ran no kernels, but zero again to be certain
+        m.counts.zero_()
     torch.cuda.synchronize()
 
     def new_event():
         return torch.cuda.Event(enable_timing=True)
 
-    with torch.cuda.stream(compute):
-        for i in range(args.warmup):
-            for g in graphs[0]:
-                g.replay()
-    torch.cuda.synchronize()
     ev_s = [new_event() for _ in range(steps)]
     ev_e = [new_event() for _ in range(steps)]
-    updates = []
+    swap_steps = set()
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
+    lag = 8   # the host stays at most this many steps ahead of the GPU, as a
+    #          serving loop that consumes each step's output does
     with torch.cuda.stream(compute):
-        for s in range(steps):
-            if s > 0 and s % epoch == 0:
-                compute.synchronize()
-                sel = hist[s - epoch:s].cpu().numpy()
-                c0, c1 = new_event(), new_event()
-                plans, n_prom, n_dem = [], 0, 0
-                with torch.cuda.stream(copy):
-                    c0.record(copy)
-                    for l in range(nl):
-                        new_hot = _hot_set(np.bincount(sel[:, l].ravel(), minlength=E), n_hot)
-                        keep = set(new_hot.tolist())
-                        promote = [e for e in new_hot.tolist() if e not in bf16[l]]
-                        demote = [e for e in hot[l].tolist() if e not in keep]
-                        fresh = {e: (host13[l][e].to(device, non_blocking=True),
-                                     host2[l][e].to(device, non_blocking=True)) for e in promote}
-                        plans.append((l, promote, demote, fresh, new_hot))
-                        n_prom += len(promote)
-                        n_dem += len(demote)
-                    c1.record(copy)
-                compute.wait_event(c1)
-                for l, promote, demote, fresh, new_hot in plans:
-                    for e in demote:
-                        q13, s13, q2, s2 = int4[l][e]
-                        layers[l].set_expert(e, B.INT4, q13, s13, q2, s2, stream=compute)
-                        del bf16[l][e]
-                    for e in promote:
-                        bf16[l][e] = fresh[e]
-                        layers[l].set_expert(e, B.BF16, fresh[e][0], None, fresh[e][1], None,
-                                             stream=compute)
-                    hot[l] = new_hot
-                prec_hist.append([np.isin(np.arange(E), hot[l]) for l in range(nl)])
-                updates.append({"step": s, "promoted": n_prom, "demoted": n_dem,
-                                "h2d_bytes": n_prom * expert_bytes(synth.BF16, H, I),
-                                "copy": (c0, c1)})
-            ev_s[s].record(compute)
-            for g in graphs[s]:
-                g.replay()
-            ev_e[s].record(compute)
+        for st in range(steps):
+            if st >= lag:
+                ev_e[st - lag].synchronize()
+            ev_s[st].record(compute)
+            for l in range(nl):
+                if mgrs[l].poll(st, compute):
+                    swap_steps.add(st)
+                if st > 0 and st % epoch == 0:
+                    mgrs[l].end_window(st, compute)
+                graphs[st][l].replay()
+            ev_e[st].record(compute)
     torch.cuda.synchronize()
     clk = clocks.stop()
     status = B.moe_get_device_status()
@@ -577,42 +546,49 @@ def stack_run(args, device, hbm_gbs, peak_src):
         raise RuntimeError(f"device status {status:#x} after the stack run")
 
     step_ms = np.array([a.elapsed_time(b) for a, b in zip(ev_s, ev_e)])
+    gaps = np.array([ev_e[i - 1].elapsed_time(ev_s[i]) for i in range(1, steps)])
     total_ms = ev_s[0].elapsed_time(ev_e[-1])
-    upd_steps = {u["step"] for u in updates}
-    for u in updates:
-        u["gap_ms"] = ev_e[u["step"] - 1].elapsed_time(ev_s[u["step"]])
-        u["copy_ms"] = u["copy"][0].elapsed_time(u["copy"][1])
-        u["h2d_gbs"] = u["h2d_bytes"] / (u["copy_ms"] * 1e-3) / 1e9 if u["copy_ms"] > 0 else None
-        del u["copy"]
     sel = hist.cpu().numpy()
+    # touched expert bytes of every step under the precision map in effect then
+    # (a swap enqueued at step s precedes that step's forwards on the stream)
     touched = np.zeros(steps)
-    for s in range(steps):
-        bf = prec_hist[s // epoch]
-        for l in range(nl):
-            te = np.unique(sel[s, l])
-            nb = int(bf[l][te].sum())
-            touched[s] += nb * expert_bytes(synth.BF16, H, I) + \
-                (len(te) - nb) * expert_bytes(synth.INT4, H, I)
-    plain = np.array([s for s in range(steps) if s not in upd_steps])
-    mean_step = float(step_ms[plain].mean())
-    gbs = float(np.mean(touched[plain] / (step_ms[plain] * 1e-3) / 1e9))
+    for l in range(nl):
+        sets = [(s_, set(d.tolist())) for s_, e_, d in mgrs[l].log if e_ in ("bootstrap", "swap")]
+        for st in range(steps):
+            hot = [h for s_, h in sets if s_ <= st][-1]
+            for e in np.unique(sel[st, l]).tolist():
+                touched[st] += expert_bytes(synth.BF16 if e in hot else synth.INT4, H, I)
+    updates = [{"layer": l, "step": s_, "event": e_} for l in range(nl)
+               for s_, e_, d in mgrs[l].log if e_ != "bootstrap"]
+    gbs = float(np.mean(touched / (step_ms * 1e-3) / 1e9))
+    mean_step = float(step_ms.mean())
+    res = {"workload": f"qwen3_80b_stack: {nl} layers x {steps} steps, H={H} I={I} E={E} "
+                       f"top-{k} T={T}, Zipf({S['zipf_s']}) popularity redrawn every {epoch} "
+                       f"steps, {n_hot} hottest BF16 per layer (device-side hot sets), every "
+                       f"expert resident as INT4",
+           "data": "synthetic (logits and x host-seeded; experts drawn on the device)",
+           "timing": "CUDA events on the compute stream; a step is one CUDA graph per layer; "
+                     "no L2 flush (a step streams hundreds of MB of experts through the L2)",
+           "tokens_per_s": T / (mean_step * 1e-3), "ms_per_step": mean_step,
+           "ms_per_layer": mean_step / nl,
+           "ms_per_step_p50": float(np.median(step_ms)),
+           "ms_per_step_max": float(step_ms.max()),
+           "tokens_per_s_with_updates": T * steps / (total_ms * 1e-3), "total_ms": total_ms,
+           "touched_bytes_per_step": float(touched.mean()),
+           "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_gbs, "peak_source": peak_src,
+           "stall_ms": {"max_gap_between_steps": float(gaps.max()),
+                        "mean_gap": float(gaps.mean()),
+                        "max_gap_at_swap_steps": float(max([gaps[s_ - 1] for s_ in swap_steps
+                                                            if s_ > 0] or [0.0]))},
+           "h2d_bytes": int(sum(m.h2d_bytes for m in mgrs)),
+           "swap_steps": sorted(swap_steps),
+           "updates": updates, "clocks": clk}
     del graphs
+    for m in mgrs:
+        m.close()
     for L in layers:
         L.close()
-    return {"workload": f"qwen3_80b_stack: {nl} layers x {steps} steps, H={H} I={I} E={E} "
-                        f"top-{k} T={T}, Zipf({S['zipf_s']}) popularity redrawn every {epoch} "
-                        f"steps, {n_hot} hottest BF16 per layer, every expert resident as INT4",
-            "data": "synthetic (logits and x host-seeded; experts drawn on the device)",
-            "timing": "CUDA events on the compute stream; a step is one CUDA graph per layer; "
-                      "no L2 flush (a step streams more than 1 GB of experts through the 126 MB L2)",
-            "tokens_per_s": T / (mean_step * 1e-3), "ms_per_step": mean_step,
-            "ms_per_layer": mean_step / nl,
-            "ms_per_step_p50": float(np.median(step_ms[plain])),
-            "ms_per_step_max": float(step_ms[plain].max()),
-            "tokens_per_s_with_updates": T * steps / (total_ms * 1e-3), "total_ms": total_ms,
-            "touched_bytes_per_step": float(touched[plain].mean()),
-            "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_gbs, "peak_source": peak_src,
-            "updates": updates, "clocks": clk}
+    return res
 
 
 # ----------------------------------------------------------------- main --
@@ -652,6 +628,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the shortened Mixtral and stack workloads of the default line")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill workload and print its object (for profiling)")
     ap.add_argument("--workload", default="decode", choices=["decode", "mixtral-sweep", "stack"],
@@ -735,6 +713,16 @@ def main():
     if not args.no_prefill:
         prefill = prefill_result(args, world, device, barrier, tf_burst, peak_src)
 
+    secondary = None
+    if not args.no_secondary:
+        # the other workloads of the layer, shortened so the default run stays
+        # within minutes: three points of the Mixtral sweep and one stack layer
+        # over two 64-step windows (one device-side hot-set update)
+        secondary = {"mixtral": mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src,
+                                              batches=(1, 32, 4096)),
+                     "stack": stack_run(args, device, hbm_gbs, peak_src, n_layers=1,
+                                        n_steps=128)}
+
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         cpu = oracle_baseline(cfg, budget_s=10.0)
@@ -765,6 +753,7 @@ def main():
             "clocks": dec["clocks"],
             "cpu_baseline": cpu,
             "prefill": prefill,
+            "secondary": secondary,
         }
         print(json.dumps(line))
     if world > 1:

@@ -80,6 +80,7 @@ constexpr long long kDrainCycles = 2000000;  // ~1 ms: bound of a wait in the gi
 constexpr int kFmaRows = 2;
 constexpr int kFmaXBytes = 2 * kFmaRows * 256;     // X of an INT4 stage (two 128-K boxes)
 constexpr int kFmaScaleBytes = 2 * kBoxRows * 2;   // fp16 scales of two K-groups
+constexpr int kFmaMinStages = 16;                  // CUDA-core units only from this K on
 constexpr int kFmaXStageMin =                      // X part of a stage, 1024-aligned
     (kFmaXBytes + kFmaScaleBytes + 1023) / 1024 * 1024;
 
@@ -456,11 +457,21 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
     un.wrow0 = wb * (kSwap ? 128 : 256);
     un.nbox = min(kSwap ? 1 : 2, (p.H - un.wrow0) / kBoxRows);
   }
-  const bool fma = kSwap && un.prec != MOE_BF16 && en.nrows <= p.fma_rows;
+  // CUDA-core units: an INT8/INT4 expert with at most fma_rows rows runs a
+  // projection on CUDA cores when its K spans at least kFmaMinStages stages.
+  // Shorter units do not repay a unit's fixed costs (first-stage latency, the
+  // output stores, the ring stages held while computing): measured on the
+  // same B200, gate/up units of K = 2048 (8 INT4 stages) were neutral at the
+  // Qwen3-30B-A3B decode shape and 6 % slower at the 512-expert stack shape,
+  // while K = 4096 / 14336 (Mixtral-8x7B shape) ran 1.3-1.8x faster.
+  const int step = un.prec == MOE_INT4 ? 256 : 128;
+  const bool fma_q = kSwap && un.prec != MOE_BF16 && en.nrows <= p.fma_rows;
+  const bool fma_gu = fma_q && p.H / step >= kFmaMinStages;
+  const bool fma = gu ? fma_gu : fma_q && p.I / step >= kFmaMinStages;
   un.flags = kUnitValid | (gu ? kUnitGateUp : 0) | (fma ? kUnitFma : 0);
   // gate/up arrivals: the 4 epilogue warps of a tensor-core unit, or every
-  // dequant warp of a CUDA-core unit (an expert's units are all of one kind)
-  un.need = (fma ? kDequantWarps : 4) * tiles_of(en.nrows, p) * p.nwb_gu;
+  // dequant warp of a CUDA-core unit
+  un.need = (fma_gu ? kDequantWarps : 4) * tiles_of(en.nrows, p) * p.nwb_gu;
   un.ent = lo;
   return un;
 }

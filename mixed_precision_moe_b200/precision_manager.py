@@ -57,7 +57,7 @@ class PrecisionManager:
         self.sel_ev = None                 # selection of the pending promotion
         self.copy_ev = None                # its copies
         self.target = None                 # set being filled
-        self.log = []                      # (step, event, details)
+        self.log = []                      # (step, event, details); swaps carry the hot ids
         self.h2d_bytes = 0
 
     # -- set-up: an initial hot set (not timed) ------------------------------
@@ -74,7 +74,7 @@ class PrecisionManager:
         self.layer.apply_hot_set(self.hot_dev[0], len(hot), 0, stream=compute)
         self.resident[0] = {e: i for i, e in enumerate(hot.tolist())}
         self.active, self.applied_hot = 0, hot
-        self.log.append((0, "bootstrap", 0))
+        self.log.append((0, "bootstrap", hot.copy()))
 
     # -- one counting window ends: select on the device ---------------------
     def end_window(self, step: int, compute):
@@ -140,7 +140,7 @@ class PrecisionManager:
         self.active = t
         self.applied_hot = self.pending_hot
         self.target, self.sel_ev, self.copy_ev = None, None, None
-        self.log.append((step, "swap", t))
+        self.log.append((step, "swap", np.sort(self.applied_hot)))
         return True
 
     def hot_experts(self):

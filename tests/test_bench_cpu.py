@@ -28,15 +28,6 @@ def test_expert_bytes_follow_the_storage_formula():
         assert bench.expert_bytes(synth.INT8, H, I) == P + 2 * (P // 128)
 
 
-def test_hot_set_takes_the_most_selected_with_ties_to_the_lower_id():
-    counts = np.array([5, 9, 5, 0, 9, 7, 5])
-    assert bench._hot_set(counts, 2).tolist() == [1, 4]
-    assert bench._hot_set(counts, 3).tolist() == [1, 4, 5]
-    assert bench._hot_set(counts, 4).tolist() == [0, 1, 4, 5]     # 5s: id 0 before 2 and 6
-    assert bench._hot_set(counts, 6).tolist() == [0, 1, 2, 4, 5, 6]
-    assert bench._hot_set(np.zeros(5, int), 2).tolist() == [0, 1]
-
-
 def test_traffic_record_is_used_only_for_the_recorded_kernel(tmp_path, monkeypatch):
     rec = tmp_path / "profile.md"
     h = bench.ffn_kernel_hash()

@@ -372,3 +372,36 @@ def test_handle_swap_is_stream_ordered():
     check_close(bf16_to_f64(out2), ref2, "after swap")
     assert layer.precision(0) == oracle.BF16 and layer.precision(1) == oracle.INT4
     layer.close()
+
+
+def test_grouped_ffn_cuda_core_units_against_oracle():
+    """INT8/INT4 experts of one or two rows whose projections span at least 16
+    CUDA-core stages (K = 4224: INT4 stages of 256 K-elements, the last one half
+    past K, read as zeros) are computed on CUDA cores from the codes; an INT4
+    expert of three rows (tensor core) and a BF16 expert share the launch.
+    Arbitrary codes (INT4 -8, INT8 -128) and quantiser codes; every expert's
+    rows equal its own launch bit for bit."""
+    H = I = 4224
+    groups = [1, 2, 2, 1, 2, 3, 1]
+    precs = [oracle.INT4, oracle.INT8, oracle.INT4, oracle.INT8, oracle.BF16, oracle.INT4,
+             oracle.INT4]
+    exps, offsets, x_perm, y_o = _ffn_case(H, I, precs, groups, 4224)
+    for e in (2, 3):   # arbitrary codes for two of the CUDA-core experts
+        ex = exps[e]
+        ex.w13, ex.s13 = synth.gen_random_codes(2 * I, H, ex.prec, 4224, 2 * e)
+        ex.w2, ex.s2 = synth.gen_random_codes(H, I, ex.prec, 4224, 2 * e + 1)
+    y_o = oracle.grouped_ffn(x_perm, offsets, exps, H, I)
+    E = len(groups)
+    layer = gpu_layer(H, I, E, E, exps)   # k = E: T = 2 tokens, swap orientation
+    xg = to_gpu_bf16(x_perm)
+    off = torch.from_numpy(offsets).cuda()
+    y = B.moe_grouped_ffn_mixed(layer, xg, off)
+    y64 = bf16_to_f64(y)
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        check_close(y64[a:b], y_o[a:b], f"expert {e} prec {precs[e]} rows {b - a}")
+        solo = np.where(np.arange(E + 1) <= e, a, b).astype(np.int32)
+        ys = B.moe_grouped_ffn_mixed(layer, xg, torch.from_numpy(solo).cuda())
+        assert torch.equal(ys[a:b].view(torch.int16), y[a:b].view(torch.int16)), f"expert {e}"
+    assert _status() == 0
+    layer.close()
