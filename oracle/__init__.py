@@ -11,6 +11,6 @@ only builds it with gcc and marshals numpy arrays through ctypes.
 """
 from .oracle import (  # noqa: F401
     BF16, INT8, INT4, build, num_threads, set_num_threads, bf16_to_double, fp16_to_double,
-    fp16_from_float, quantize, dequantize, route_topk, permute, grouped_ffn,
+    fp16_from_float, quantize, dequantize, router_logits, route_topk, permute, grouped_ffn,
     combine, moe_layer, Expert, seeded_experts,
 )

@@ -11,6 +11,7 @@
  * What it computes, with the passage each step follows (page "Every Expert
  * Counts: ExactMoE for Memory-Efficient W4A16 Inference", arXiv 2608.15383):
  *
+ *   router   z_t = W_r h_t, bf16 operands, binary64 sum          -- Section 3.1, routing equation
  *   route    S_t = TopK(z_t, k) over the router logits        -- Section 3.1, routing equation
  *            ties between equal logits go to the lower expert id (the top-k
  *            rule is "unchanged" and must be deterministic); the gating weights
@@ -202,6 +203,27 @@ int oracle_quantize(const uint16_t* w, int rows, int K, int prec, void* q_out,
 /* ------------------------------------------------------------------------ */
 /* Routing (Section 3.1 routing equation)                                    */
 /* ------------------------------------------------------------------------ */
+
+/* Router projection z_t = W_r h_t (Section 3.1 routing equation; the router
+ * stays in BF16, Abstract): h bf16 [T][H] (one hidden state per token), wr
+ * bf16 [E][H] (row e = expert e's router row) -> z [T][E] in binary64.  Every
+ * bf16 value and every product of two is exact in binary64; the products are
+ * summed in ascending hidden index. */
+int oracle_router_logits(const uint16_t* h, const uint16_t* wr, int T, int H, int E,
+                         double* z) {
+  if (T < 0 || H <= 0 || E <= 0) return OR_ERR_ARG;
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < T; ++t) {
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int c = 0; c < H; ++c)
+        acc += oracle_bf16_to_double(h[(size_t)t * H + c]) *
+               oracle_bf16_to_double(wr[(size_t)e * H + c]);
+      z[(size_t)t * E + e] = acc;
+    }
+  }
+  return OR_OK;
+}
 
 /* logits fp32 [T][E]. Writes idx [T][k] (descending logit, ties -> lower id)
  * and weights [T][k] in binary64.  renormalize != 0: softmax over the k

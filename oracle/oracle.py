@@ -103,6 +103,20 @@ def dequantize(prec: int, w: np.ndarray, s: np.ndarray | None, rows: int, K: int
     return out
 
 
+def router_logits(h: np.ndarray, wr: np.ndarray) -> np.ndarray:
+    """z = W_r h per token in binary64 (ExactMoE Section 3.1 routing equation).
+    h: bf16 bit patterns uint16 [T][H]; wr: uint16 [E][H]."""
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    wr = np.ascontiguousarray(wr, dtype=np.uint16)
+    T, H = h.shape
+    E, H2 = wr.shape
+    if H2 != H:
+        raise ValueError("router rows must have the hidden size")
+    z = np.zeros((T, E), np.float64)
+    _check(_L().oracle_router_logits(_p(h), _p(wr), T, H, E, _p(z)), "router")
+    return z
+
+
 def route_topk(logits: np.ndarray, k: int, renormalize: bool = True):
     z = np.ascontiguousarray(logits, dtype=np.float32)
     T, E = z.shape

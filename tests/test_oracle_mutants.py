@@ -55,6 +55,10 @@ MUTANTS = {
                            "if (idx[(size_t)t * k + jj] == e + E) return 1;"),
     "layer_weight_slot": ("double wj = w[(size_t)t * k + j];\n          for (int c = 0; c < H; ++c) o[c] += wj * y[c];",
                           "double wj = w[(size_t)t * k + (j + 1) % k];\n          for (int c = 0; c < H; ++c) o[c] += wj * y[c];"),
+    "router_transposed": ("oracle_bf16_to_double(wr[(size_t)e * H + c]);",
+                          "oracle_bf16_to_double(wr[(size_t)c * E + e]);"),
+    "router_drops_last_column": ("for (int c = 0; c < H; ++c)\n        acc +=",
+                                 "for (int c = 0; c < H - 1; ++c)\n        acc +="),
     "combine_weight_slot": ("double wj = w[(size_t)t * k + j];\n      for (int c = 0; c < H; ++c) o[c] += wj * y_perm",
                             "double wj = w[(size_t)t * k + (j + 1) % k];\n      for (int c = 0; c < H; ++c) o[c] += wj * y_perm"),
 }

@@ -54,6 +54,63 @@ def test_bf16_to_double_matches_torch():
     assert np.array_equal(got, ref)
 
 
+# ------------------------------------------------------- router projection --
+
+def _bf16_bits(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).view(torch.int16) \
+        .numpy().view(np.uint16)
+
+
+def _bf16_values(bits):
+    return torch.from_numpy(np.asarray(bits, np.uint16).view(np.int16)).view(torch.bfloat16) \
+        .double().numpy()
+
+
+@pytest.mark.parametrize("T,H,E", [(5, 256, 8), (33, 384, 128), (3, 2048, 17), (0, 128, 4)])
+def test_router_logits_match_numpy_fp64_matmul(T, H, E):
+    # z = W_r h (routing equation): numpy's fp64 product of the bf16 values;
+    # the products are exact, only the summation order differs
+    rng = np.random.default_rng(T * 1000 + E)
+    h = _bf16_bits(rng.standard_normal((T, H)))
+    wr = _bf16_bits(rng.standard_normal((E, H)) * 0.02)
+    z = oracle.router_logits(h, wr)
+    ref = _bf16_values(h) @ _bf16_values(wr).T
+    assert z.shape == (T, E)
+    bound = H * 2.0 ** -52 * (np.abs(_bf16_values(h)) @ np.abs(_bf16_values(wr)).T)
+    assert np.all(np.abs(z - ref) <= bound)
+
+
+def test_router_one_hot_rows_select_hidden_entries():
+    # row e of W_r = unit vector at column j_e  =>  z[t][e] = h[t][j_e] exactly
+    rng = np.random.default_rng(3)
+    T, H, E = 7, 256, 16
+    h = _bf16_bits(rng.standard_normal((T, H)))
+    cols = rng.permutation(H)[:E]
+    w = np.zeros((E, H), np.float32)
+    w[np.arange(E), cols] = 1.0
+    z = oracle.router_logits(h, _bf16_bits(w))
+    assert np.array_equal(z, _bf16_values(h)[:, cols])
+
+
+def test_router_integer_inputs_are_exact_and_tie():
+    # small integers: every partial sum is an exact integer, checked against
+    # Python's own integer arithmetic; the ties this produces are then broken
+    # to the lower id by the top-k
+    rng = np.random.default_rng(4)
+    T, H, E = 6, 128, 12
+    hi = rng.integers(-2, 3, (T, H))
+    wi = rng.integers(-1, 2, (E, H))
+    wi[5] = wi[2]                      # experts 2 and 5 tie on every token
+    z = oracle.router_logits(_bf16_bits(hi), _bf16_bits(wi))
+    exact = np.array([[sum(int(a) * int(b) for a, b in zip(hi[t], wi[e])) for e in range(E)]
+                      for t in range(T)])
+    assert np.array_equal(z, exact.astype(np.float64))
+    idx, _ = oracle.route_topk(z.astype(np.float32), E)
+    for t in range(T):
+        order = idx[t].tolist()
+        assert order.index(2) < order.index(5)
+
+
 # ---------------------------------------------------------------- routing --
 
 def _brute_topk(z, k):
