@@ -430,6 +430,53 @@ def mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src, batches=None):
             "points": points, "clocks": clk}
 
 
+ROUTER_CASES = [  # name, T, H, E, k, zipf_s
+    ("qwen3_30b_decode", 32, 2048, 128, 8, 1.1),
+    ("qwen3_30b_prefill", 4096, 2048, 128, 8, 1.1),
+    ("qwen3_80b_stack_layer", 32, 2048, 512, 10, 1.2),
+    ("mixtral_8x7b_t1", 1, 4096, 8, 2, 0.0),
+    ("mixtral_8x7b_t4096", 4096, 4096, 8, 2, 0.0),
+]
+
+
+def router_run(args, device, hbm_gbs, peak_src):
+    """The router projection fused with top-k (moe_router_topk, one launch) on
+    the layers' shapes: time per launch and its bytes (h, W_r, the top-k
+    outputs) against HBM, from CUDA-graph replays with L2 flushed between."""
+    from mixed_precision_moe_b200 import binding as B
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    steps, warmup = max(20, args.steps // 4), args.warmup
+    points = []
+    for name, T, H, E, k, zs in ROUTER_CASES:
+        hb, wb = synth.gen_router(T, H, E, 900 + T + E, zs)
+        h = torch.from_numpy(hb.view(np.int16)).view(torch.bfloat16).to(device)
+        wr = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(device)
+        idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        w = torch.empty((T, k), dtype=torch.float32, device=device)
+        with torch.cuda.stream(stream):
+            B.moe_router_topk(h, wr, k, topk_idx=idx, topk_w=w, stream=stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            B.moe_router_topk(h, wr, k, topk_idx=idx, topk_w=w, stream=stream)
+        ms = float(np.mean(time_graphs([g], steps, warmup, flush, stream)))
+        nbytes = 2 * T * H + 2 * E * H + 8 * T * k
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        points.append({"workload": name, "T": T, "H": H, "E": E, "k": k, "us": ms * 1e3,
+                       "tokens_per_s": T / (ms * 1e-3), "bytes": nbytes, "achieved_gbs": gbs,
+                       "frac_hbm": gbs / hbm_gbs, "tflops": 2.0 * T * E * H / (ms * 1e-3) / 1e12})
+        del g
+    status = B.moe_get_device_status()
+    if status:
+        raise RuntimeError(f"device status {status:#x} after the router runs")
+    return {"kernel": "router_topk_kernel (z = W_r h on tcgen05, K split over a cluster, "
+                      "top-k in the epilogue)",
+            "timing": f"CUDA graph of one launch, {steps} timed replays after {warmup}, "
+                      "L2 flushed between",
+            "peaks": {"hbm_gbs": hbm_gbs, "source": peak_src}, "points": points}
+
+
 def stack_run(args, device, hbm_gbs, peak_src, n_layers=None, n_steps=None):
     """Qwen3-80B-scale stack: layers of H 2048, I 512, 512 experts, top-10 at
     decode batch 32, Zipf(1.2) routing whose popularity order is redrawn every
@@ -632,8 +679,9 @@ def main():
                     help="skip the shortened Mixtral and stack workloads of the default line")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill workload and print its object (for profiling)")
-    ap.add_argument("--workload", default="decode", choices=["decode", "mixtral-sweep", "stack"],
-                    help="decode: the headline line; mixtral-sweep / stack: one JSON object "
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "mixtral-sweep", "stack", "router"],
+                    help="decode: the headline line; mixtral-sweep / stack / router: one JSON object "
                          "for that workload instead (one GPU)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -691,6 +739,8 @@ def main():
             raise SystemExit(f"--workload {args.workload} runs on one GPU")
         if args.workload == "mixtral-sweep":
             print(json.dumps(mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src)))
+        elif args.workload == "router":
+            print(json.dumps(router_run(args, device, hbm_gbs, peak_src)))
         else:
             print(json.dumps(stack_run(args, device, hbm_gbs, peak_src)))
         return
@@ -721,7 +771,8 @@ def main():
         secondary = {"mixtral": mixtral_sweep(args, device, hbm_gbs, tf_burst, peak_src,
                                               batches=(1, 32, 4096)),
                      "stack": stack_run(args, device, hbm_gbs, peak_src, n_layers=1,
-                                        n_steps=128)}
+                                        n_steps=128),
+                     "router": router_run(args, device, hbm_gbs, peak_src)}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:

@@ -120,6 +120,24 @@ int moe_get_expert_precision(moe_layer_t layer, int expert, int* precision);
 int moe_route_topk(const float* logits, int T, int E, int k, int renormalize,
                    int32_t* topk_idx, float* topk_w, void* stream);
 
+/* Router projection fused with top-k routing (ExactMoE Section 3.1 routing
+ * equation z_t = W_r h_t, S_t = TopK(z_t, k); the router stays in BF16,
+ * Abstract):
+ *   h          device bf16 [T][H], the layer's input hidden states, row-major
+ *   w_router   device bf16 [E][H], row e = expert e's router weights
+ *   logits     device fp32 [T][E] or NULL: z in fp32 (bf16 products summed in
+ *              fp32 on the tensor cores; the K split is summed in a fixed
+ *              order, so results are deterministic)
+ *   topk_idx, topk_w: as moe_route_topk, computed from those fp32 logits with
+ *              the same rule (identical to moe_route_topk on `logits`)
+ * H a multiple of 64, 1 <= E <= 512, 1 <= k <= min(E, 16); h and w_router
+ * 16-byte aligned.  One launch: a thread-block cluster splits each tile of
+ * tokens' K range over up to 8 CTAs, reduces the partial logits through
+ * distributed shared memory and routes the tile's tokens. */
+int moe_router_topk(const void* h, const void* w_router, int T, int H, int E, int k,
+                    int renormalize, float* logits, int32_t* topk_idx, float* topk_w,
+                    void* stream);
+
 /* Group the T*k (token, slot) pairs by expert (ExactMoE Figure 1), experts in
  * id order, ascending token inside each expert; no pair is dropped.
  *   topk_idx       device int32 [T][k]; ids must lie in [0,E) and be distinct
@@ -224,6 +242,20 @@ int moe_layer_forward(moe_layer_t layer, const float* logits, const void* x, int
                       int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row,
                       void* x_perm, void* y_perm, void* workspace, size_t workspace_bytes,
                       void* out, void* stream);
+
+/* The whole layer from the hidden states: z = W_r x (moe_router_topk) ->
+ * top-k -> moe_permute -> moe_grouped_ffn_mixed -> moe_combine, the same
+ * buffers as moe_layer_forward except that `logits` (fp32 [T][E]) is written
+ * (the router's output) instead of read, and w_router (bf16 [E][H], the
+ * layer's H and E) is added.  The outputs equal moe_layer_forward's on the
+ * logits this call writes.  For T <= 128 the router kernel writes the logits
+ * and the small-batch kernel routes them; above, the router kernel also takes
+ * the top-k. */
+int moe_layer_forward_hidden(moe_layer_t layer, const void* x, const void* w_router, int T,
+                             int renormalize, float* logits, int32_t* topk_idx, float* topk_w,
+                             int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row,
+                             void* x_perm, void* y_perm, void* workspace, size_t workspace_bytes,
+                             void* out, void* stream);
 
 /* Symmetric group-128 quantiser (ExactMoE Section 3.2; INT8 by analogy with
  * Q = 127): for each row and K-group g, s = fp16_rne(max|W| / Q) with the

@@ -31,6 +31,7 @@ SIGNATURES = {
     "moe_set_expert_precision": (_I, [_P, _I, _I, _P, _P]),
     "moe_get_expert_precision": (_I, [_P, _I, C.POINTER(_I)]),
     "moe_route_topk": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
+    "moe_router_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "moe_permute": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_ffn_workspace_bytes": (_I, [_P, _I, C.POINTER(_S)]),
     "moe_grouped_ffn_mixed": (_I, [_P, _P, _P, _I, _P, _P, _S, _P]),
@@ -39,6 +40,8 @@ SIGNATURES = {
     "moe_ffn_noalloc_reset": (_I, []),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_layer_forward": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _P]),
+    "moe_layer_forward_hidden": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S,
+                                      _P, _P]),
     "moe_quantize_weights": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "moe_get_device_status": (_I, [C.POINTER(C.c_uint)]),
     "moe_layer_set_hotness_counter": (_I, [_P, _P]),
@@ -110,6 +113,29 @@ def moe_route_topk(logits, k, renormalize=True, topk_idx=None, topk_w=None, stre
         topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
     _check(lib().moe_route_topk(_ptr(logits), T, E, k, int(bool(renormalize)), _ptr(topk_idx),
                                 _ptr(topk_w), _stream(stream)))
+    return topk_idx, topk_w
+
+
+def moe_router_topk(h, w_router, k, renormalize=True, logits=None, topk_idx=None, topk_w=None,
+                    stream=None):
+    """z = W_r h (fp32, written to `logits` if given) and its top-k; returns
+    (topk_idx [T,k] int32, topk_w [T,k] fp32)."""
+    _need(h, torch.bfloat16, "h")
+    _need(w_router, torch.bfloat16, "w_router")
+    T, H = h.shape
+    E = w_router.shape[0]
+    if w_router.shape[1] != H:
+        raise ValueError("w_router must be [E, H]")
+    if logits is not None:
+        _need(logits, torch.float32, "logits")
+        if tuple(logits.shape) != (T, E):
+            raise ValueError("logits must be [T, E]")
+    if topk_idx is None:
+        topk_idx = torch.empty((T, k), dtype=torch.int32, device=h.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=h.device)
+    _check(lib().moe_router_topk(_ptr(h), _ptr(w_router), T, H, E, k, int(bool(renormalize)),
+                                 _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
     return topk_idx, topk_w
 
 
@@ -303,6 +329,27 @@ class MoELayer:
                                        _stream(stream)))
         return out
 
+    def forward_hidden(self, x, w_router, renormalize=True, bufs=None, stream=None):
+        """router (z = W_r x) -> route -> permute -> grouped FFN -> combine (one
+        moe_layer_forward_hidden call); returns out [T, H] bf16.  The logits
+        land in bufs["logits"]."""
+        _need(x, torch.bfloat16, "x")
+        _need(w_router, torch.bfloat16, "w_router")
+        if tuple(w_router.shape) != (self.E, self.H):
+            raise ValueError("w_router must be [E, H]")
+        T = x.shape[0]
+        if bufs is None:
+            bufs = self.alloc_buffers(T, x.device)
+        idx, w = bufs["route"]
+        off, perm, dest, xp = bufs["permute"]
+        y, ws = bufs["ffn"]
+        out = bufs["out"]
+        _check(lib().moe_layer_forward_hidden(
+            self.handle, _ptr(x), _ptr(w_router), T, int(bool(renormalize)), _ptr(bufs["logits"]),
+            _ptr(idx), _ptr(w), _ptr(off), _ptr(perm), _ptr(dest), _ptr(xp), _ptr(y), _ptr(ws),
+            ws.numel(), _ptr(out), _stream(stream)))
+        return out
+
     def alloc_buffers(self, T, device="cuda"):
         """Preallocated intermediates for forward(bufs=...), e.g. for graph capture."""
         k, H, E = self.k, self.H, self.E
@@ -318,6 +365,7 @@ class MoELayer:
                     torch.empty(moe_ffn_workspace_bytes(self, R), dtype=torch.uint8,
                                 device=device)),
             "out": torch.empty((T, H), dtype=torch.bfloat16, device=device),
+            "logits": torch.empty((T, E), dtype=torch.float32, device=device),
         }
 
     def close(self):

@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "grouped_ffn.cuh"
 #include "route_permute_combine.cuh"
+#include "router.cuh"
 
 namespace {
 constexpr int kMaxDevices = 64;  // per-device caches below
@@ -331,6 +332,122 @@ int moe_route_topk(const float* logits, int T, int E, int k, int renormalize, in
   return ok();
 }
 
+}  // extern "C"
+
+namespace {
+// ------------------------------------------------ router projection + top-k --
+// Host checks of moe_router_topk's arguments (also run by
+// moe_layer_forward_hidden before it enqueues anything).
+int router_check(const void* h, const void* w_router, int T, int H, int E, int k, int do_topk,
+                 const float* logits, const int32_t* topk_idx, const float* topk_w) {
+  MOE_CHECK(T >= 0, MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  MOE_CHECK(H >= moe::router::kKB && H % moe::router::kKB == 0, MOE_ERR_UNSUPPORTED,
+            "H=%d must be a positive multiple of %d", H, moe::router::kKB);
+  MOE_CHECK(E >= 1 && E <= moe::router::kMaxE, MOE_ERR_UNSUPPORTED, "E=%d outside [1, 512]", E);
+  if (do_topk)
+    MOE_CHECK(k >= 1 && k <= 16 && k <= E, MOE_ERR_INVALID_ARG, "k=%d outside [1, min(E, 16)]",
+              k);
+  MOE_CHECK((T + moe::router::tm_of(E) - 1) / moe::router::tm_of(E) <= 65535,
+            MOE_ERR_UNSUPPORTED, "T=%d too large", T);
+  if (T == 0) return MOE_OK;
+  MOE_CHECK(h && w_router, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_CHECK(!do_topk || (topk_idx && topk_w), MOE_ERR_INVALID_ARG, "null top-k output");
+  MOE_CHECK(do_topk || logits, MOE_ERR_INVALID_ARG, "nothing to write: no logits, no top-k");
+  MOE_CHECK(aligned(h, 16) && aligned(w_router, 16), MOE_ERR_UNSUPPORTED,
+            "h and w_router must be 16-byte aligned");
+  return MOE_OK;
+}
+
+template <int KEYS>
+int router_launch(const CUtensorMap& tm_h, const CUtensorMap& tm_w, const moe::router::Params& prm,
+                  int S, int tiles, size_t smem, int dev, cudaStream_t s) {
+  static std::atomic<bool> done[kMaxDevices];
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (!(cached && done[dev].load())) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(moe::router::router_topk_kernel<KEYS>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)moe::router::kSmemLimit));
+    if (cached) done[dev].store(true);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S, tiles);
+  cfg.blockDim = dim3(moe::router::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, moe::router::router_topk_kernel<KEYS>, tm_h, tm_w, prm));
+  return MOE_OK;
+}
+
+// z = W_r h on the tensor cores, then (do_topk) the top-k of every token.
+// Cluster size S: the largest power of two <= 8 (and <= H / 64) that keeps
+// tiles * S within the SM count; stages: as many as the shared memory holds,
+// up to the k-blocks of one CTA.
+int router_impl(const void* h, const void* w_router, int T, int H, int E, int k, int renormalize,
+                int do_topk, float* logits, int32_t* topk_idx, float* topk_w, void* stream) {
+  namespace R = moe::router;
+  int rc = router_check(h, w_router, T, H, E, k, do_topk, logits, topk_idx, topk_w);
+  if (rc != MOE_OK || T == 0) return rc;
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  const int npad = R::npad_of(E), tm = R::tm_of(E), nkb = H / R::kKB;
+  const int tiles = (T + tm - 1) / tm;
+  const int nsm = std::max(1, num_sms(dev));
+  int S = 1;
+  while (S * 2 <= R::kMaxCluster && S * 2 <= nkb && tiles * S * 2 <= nsm) S *= 2;
+  const int nkl_max = (nkb + S - 1) / S;
+  int ns = 1;
+  while (ns < nkl_max && R::layout(npad, tm, ns + 1, S).total <= R::kSmemLimit) ++ns;
+  const size_t smem = R::layout(npad, tm, ns, S).total;
+  MOE_CHECK(smem <= R::kSmemLimit, MOE_ERR_UNSUPPORTED, "router tile does not fit (E=%d)", E);
+  CUtensorMap tm_h, tm_w;
+  rc = encode_2d(&tm_h, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, H, tm, R::kKB,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != MOE_OK) return rc;
+  rc = encode_2d(&tm_w, w_router, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, H, std::min(npad, 256),
+                 R::kKB, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != MOE_OK) return rc;
+  R::Params prm;
+  prm.T = T;
+  prm.H = H;
+  prm.E = E;
+  prm.k = k;
+  prm.renormalize = renormalize;
+  prm.do_topk = do_topk;
+  prm.npad = npad;
+  prm.tm = tm;
+  prm.nkb = nkb;
+  prm.ns = ns;
+  prm.logits = logits;
+  prm.topk_idx = topk_idx;
+  prm.topk_w = topk_w;
+  const int keys = (E + 31) / 32;
+  cudaStream_t s = as_stream(stream);
+  rc = keys <= 1   ? router_launch<1>(tm_h, tm_w, prm, S, tiles, smem, dev, s)
+       : keys <= 2 ? router_launch<2>(tm_h, tm_w, prm, S, tiles, smem, dev, s)
+       : keys <= 4 ? router_launch<4>(tm_h, tm_w, prm, S, tiles, smem, dev, s)
+       : keys <= 8 ? router_launch<8>(tm_h, tm_w, prm, S, tiles, smem, dev, s)
+                   : router_launch<16>(tm_h, tm_w, prm, S, tiles, smem, dev, s);
+  return rc;
+}
+}  // namespace
+
+extern "C" {
+int moe_router_topk(const void* h, const void* w_router, int T, int H, int E, int k,
+                    int renormalize, float* logits, int32_t* topk_idx, float* topk_w,
+                    void* stream) {
+  const int rc = router_impl(h, w_router, T, H, E, k, renormalize, 1, logits, topk_idx, topk_w,
+                             stream);
+  return rc == MOE_OK ? ok() : rc;
+}
 }  // extern "C"
 
 namespace {
@@ -660,10 +777,16 @@ int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w
   return ok();
 }
 
-int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, int renormalize,
-                      int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
-                      int32_t* perm_token, int32_t* dest_row, void* x_perm, void* y_perm,
-                      void* workspace, size_t workspace_bytes, void* out, void* stream) {
+}  // extern "C"
+
+namespace {
+// moe_layer_forward and moe_layer_forward_hidden.  w_router == NULL: the
+// logits are an input; otherwise they are computed here (z = W_r x) into
+// `logits`, and for T > 128 the router kernel also takes the top-k.
+int layer_forward_impl(moe_layer_t L, float* logits, const void* x, const void* w_router, int T,
+                       int renormalize, int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                       int32_t* perm_token, int32_t* dest_row, void* x_perm, void* y_perm,
+                       void* workspace, size_t workspace_bytes, void* out, void* stream) {
   MOE_CHECK(L != nullptr, MOE_ERR_INVALID_ARG, "layer is null");
   MOE_CHECK(T >= 0, MOE_ERR_INVALID_ARG, "T=%d < 0", T);
   if (T == 0) {  // as the separate calls: no rows, every expert empty
@@ -680,9 +803,18 @@ int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, 
             MOE_ERR_INVALID_ARG, "null pointer");
   MOE_CHECK(aligned(x, 16) && aligned(out, 16), MOE_ERR_UNSUPPORTED,
             "x and out must be 16-byte aligned");
+  if (w_router != nullptr) {
+    rc = router_check(x, w_router, T, L->H, L->E, L->k, 1, logits, topk_idx, topk_w);
+    if (rc != MOE_OK) return rc;
+  }
   if (T <= moe::kFrontMaxTokens) {
     // Small batch: routing, grouping and the row gather in one launch, which
-    // also zeroes the FFN's scheduler counters.
+    // also zeroes the FFN's scheduler counters (after the router's logits).
+    if (w_router != nullptr) {
+      rc = router_impl(x, w_router, T, L->H, L->E, L->k, renormalize, 0, logits, nullptr,
+                       nullptr, stream);
+      if (rc != MOE_OK) return rc;
+    }
     rc = route_permute_gather_small(L, logits, x, T, renormalize, topk_idx, topk_w,
                                     expert_offsets, perm_token, dest_row, x_perm, workspace,
                                     workspace_bytes, stream);
@@ -693,7 +825,11 @@ int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, 
     moe_ffn_workspace_bytes(L, T * L->k, &need);
     MOE_CUDA_TRY(cudaMemsetAsync(static_cast<uint8_t*>(workspace) + need - kFfnCounterBytes, 0,
                                  ffn_counter_bytes(L->E), as_stream(stream)));
-    rc = moe_route_topk(logits, T, L->E, L->k, renormalize, topk_idx, topk_w, stream);
+    if (w_router != nullptr)
+      rc = router_impl(x, w_router, T, L->H, L->E, L->k, renormalize, 1, logits, topk_idx, topk_w,
+                       stream);
+    else
+      rc = moe_route_topk(logits, T, L->E, L->k, renormalize, topk_idx, topk_w, stream);
     if (rc != MOE_OK) return rc;
     rc = permute_impl(topk_idx, x, T, L->E, L->k, L->H, expert_offsets, perm_token, dest_row,
                       x_perm, L->hot, stream);
@@ -703,6 +839,28 @@ int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, 
                         stream, false);
   if (rc != MOE_OK) return rc;
   return moe_combine(y_perm, dest_row, topk_w, T, L->k, L->H, out, stream);
+}
+}  // namespace
+
+extern "C" {
+int moe_layer_forward(moe_layer_t L, const float* logits, const void* x, int T, int renormalize,
+                      int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                      int32_t* perm_token, int32_t* dest_row, void* x_perm, void* y_perm,
+                      void* workspace, size_t workspace_bytes, void* out, void* stream) {
+  return layer_forward_impl(L, const_cast<float*>(logits), x, nullptr, T, renormalize, topk_idx,
+                            topk_w, expert_offsets, perm_token, dest_row, x_perm, y_perm,
+                            workspace, workspace_bytes, out, stream);
+}
+
+int moe_layer_forward_hidden(moe_layer_t L, const void* x, const void* w_router, int T,
+                             int renormalize, float* logits, int32_t* topk_idx, float* topk_w,
+                             int32_t* expert_offsets, int32_t* perm_token, int32_t* dest_row,
+                             void* x_perm, void* y_perm, void* workspace, size_t workspace_bytes,
+                             void* out, void* stream) {
+  MOE_CHECK(w_router != nullptr || T == 0, MOE_ERR_INVALID_ARG, "w_router is null");
+  return layer_forward_impl(L, logits, x, w_router, T, renormalize, topk_idx, topk_w,
+                            expert_offsets, perm_token, dest_row, x_perm, y_perm, workspace,
+                            workspace_bytes, out, stream);
 }
 
 int moe_quantize_weights(const void* w_bf16, int rows, int K, moe_precision_t precision,

@@ -58,6 +58,24 @@ def gen_logits(T: int, E: int, seed: int, zipf_s: float = 0.0,
     return np.ascontiguousarray(z, dtype=np.float32)
 
 
+def gen_router(T: int, H: int, E: int, seed: int, zipf_s: float = 0.0,
+               ranks: np.ndarray | None = None):
+    """Hidden states h bf16 bits [T, H] and router weights W_r bf16 bits
+    [E, H] for z = W_r h.  h ~N(0, 1) and W_r ~N(0, 1/H), so that z is about
+    N(0, 1) like gen_logits.  With zipf_s, the last hidden coordinate is the
+    constant 1 and W_r[e, H-1] = -zipf_s * ln(rank_e) (bf16-rounded): the
+    Zipf popularity bias of gen_logits carried by the weights, since a
+    router has no bias term of its own."""
+    h = _rng(seed, 5).standard_normal((T, H), dtype=np.float32)
+    w = _rng(seed, 6).standard_normal((E, H), dtype=np.float32) * np.float32(1.0 / np.sqrt(H))
+    if zipf_s:
+        if ranks is None:
+            ranks = zipf_ranks(E, seed)
+        h[:, H - 1] = 1.0
+        w[:, H - 1] = (-zipf_s * np.log(ranks.astype(np.float64))).astype(np.float32)
+    return to_bf16_bits(h), to_bf16_bits(w)
+
+
 def gen_expert_master(H: int, I: int, seed: int, e: int, std: float = 0.02):
     """bf16 master weights of expert e: (w13 [2I, H], w2 [H, I]) as bf16 bits.
 

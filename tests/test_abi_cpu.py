@@ -64,6 +64,15 @@ def test_host_validation_before_any_cuda_call(lib):
     assert lib.moe_route_topk(None, 4, 600, 2, 1, None, None, None) == -2
     assert lib.moe_route_topk(None, 4, 8, 2, 1, None, None, None) == -1   # null pointers
     assert lib.moe_route_topk(None, 0, 8, 2, 1, None, None, None) == 0    # T = 0: nothing to do
+    # router projection + top-k: H a multiple of 64, E <= 512, k <= min(E, 16)
+    assert lib.moe_router_topk(None, None, 4, 100, 8, 2, 1, None, None, None, None) == -2
+    assert lib.moe_router_topk(None, None, 4, 256, 513, 2, 1, None, None, None, None) == -2
+    assert lib.moe_router_topk(None, None, 4, 256, 8, 9, 1, None, None, None, None) == -1
+    assert lib.moe_router_topk(None, None, -1, 256, 8, 2, 1, None, None, None, None) == -1
+    assert lib.moe_router_topk(None, None, 4, 256, 8, 2, 1, None, None, None, None) == -1
+    assert lib.moe_router_topk(None, None, 0, 256, 8, 2, 1, None, None, None, None) == 0
+    assert lib.moe_layer_forward_hidden(None, None, None, 4, 1, None, None, None, None, None,
+                                        None, None, None, None, 0, None, None) == -1
     assert lib.moe_permute(None, None, 4, 0, 2, 256, None, None, None, None, None) == -2
     assert lib.moe_permute(None, None, 4, 8, 2, 100, None, None, None, None, None) == -2
     assert lib.moe_combine(None, None, None, 4, 0, 256, None, None) == -1
