@@ -430,7 +430,7 @@ __device__ void build_entries(const Params& p, const Smem& s, int my_prec) {
   }
 }
 
-template <bool kSwap>
+template <bool kSwap, bool kFma>
 __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int u) {
   const bool gu = u < *s.n_units_gu;
   int lo = 0, hi = *s.n_entries - 1;  // last entry whose first unit is <= u
@@ -465,7 +465,7 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
   // Qwen3-30B-A3B decode shape and 6 % slower at the 512-expert stack shape,
   // while K = 4096 / 14336 (Mixtral-8x7B shape) ran 1.3-1.8x faster.
   const int step = un.prec == MOE_INT4 ? 256 : 128;
-  const bool fma_q = kSwap && un.prec != MOE_BF16 && en.nrows <= p.fma_rows;
+  const bool fma_q = kFma && kSwap && un.prec != MOE_BF16 && en.nrows <= p.fma_rows;
   const bool fma_gu = fma_q && p.H / step >= kFmaMinStages;
   const bool fma = gu ? fma_gu : fma_q && p.I / step >= kFmaMinStages;
   un.flags = kUnitValid | (gu ? kUnitGateUp : 0) | (fma ? kUnitFma : 0);
@@ -505,14 +505,21 @@ __device__ __forceinline__ void load_scale_box(void* dst, const Params& p, const
   }
 }
 
-__device__ __forceinline__ bool unit_fma(const Unit& un) { return (un.flags & kUnitFma) != 0; }
+// kFma: the kernel instance has the CUDA-core path.  Without it every CUDA-core
+// branch is compiled out: its mere presence (code size, register allocation
+// of the roles) cost 7 % of the decode step at shapes that never use it.
+template <bool kFma>
+__device__ __forceinline__ bool unit_fma(const Unit& un) {
+  return kFma && (un.flags & kUnitFma) != 0;
+}
 
 // Operand-ring stages of a unit: one per 64-element k-block, or for a CUDA-core
 // unit one per 128 code bytes of a row (INT4: 256 K-elements, INT8: 128); the
 // last CUDA-core stage may run past K and reads zeros there (TMA fill).
+template <bool kFma>
 __device__ __forceinline__ int unit_nkb(const Params& p, const Unit& un) {
   const int K = unit_gu(un) ? p.H : p.I;
-  if (unit_fma(un)) {
+  if (unit_fma<kFma>(un)) {
     const int step = un.prec == MOE_INT4 ? 256 : 128;
     return (K + step - 1) / step;
   }
@@ -574,7 +581,7 @@ __device__ __forceinline__ bool wait_gate_up(const Params& p, const Unit& un,
 // few k-blocks before unit n's last copies: every global round trip of a unit
 // switch happens here, off the producer's path, while the late reservation
 // keeps the dynamic balance of the tail.
-template <bool kSwap>
+template <bool kSwap, bool kFma>
 __device__ void scheduler(const Params& p, const Smem& s) {
   volatile int* abort_flag = s.abort_flag;
   const int total = *s.n_units;
@@ -662,9 +669,9 @@ __device__ void scheduler(const Params& p, const Smem& s) {
     }
     Unit un = Unit{0, 0, 0, 0, 0, 0, 0, 0, 0};
     if (u < total) {
-      un = decode_unit<kSwap>(p, s, u);
+      un = decode_unit<kSwap, kFma>(p, s, u);
       const ExpertDesc* d = p.descs + un.e;
-      if (unit_fma(un))
+      if (unit_fma<kFma>(un))
         prefetch_tmap(unit_gu(un) ? &d->tm_q13f : &d->tm_q2f);
       else
         prefetch_tmap(unit_gu(un) ? &d->tm_w13 : &d->tm_w2);
@@ -693,7 +700,7 @@ __device__ void scheduler(const Params& p, const Smem& s) {
 // ---------------------------------------------------------------- producer --
 // Streams, per k-block, the X tile (one copy) and, for BF16 units, the
 // weight boxes into the operand ring.
-template <bool kSwap>
+template <bool kSwap, bool kFma>
 __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h,
                          const CUtensorMap* tm_xf, const CUtensorMap* tm_hf, const Params& p,
                          const Smem& s) {
@@ -726,7 +733,7 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h,
     FFN_TRACE_SET(tseq, kTrProdBeg, FFN_TRACE_NS());
 
     const bool gu = unit_gu(un);
-    const bool fma = kSwap && unit_fma(un);
+    const bool fma = kSwap && unit_fma<kFma>(un);
     const bool int4 = un.prec == MOE_INT4;
     const ExpertDesc* d = p.descs + un.e;
     const CUtensorMap* tw = fma ? (gu ? &d->tm_q13f : &d->tm_q2f) : (gu ? &d->tm_w13 : &d->tm_w2);
@@ -736,7 +743,7 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h,
     if (bf16 || fma) tmap_acquire(tw);
     if (fma) tmap_acquire(tsc);
     if (!gu) fence_proxy_async_global();  // h rows published (scheduler's acquire) -> TMA reads
-    const int nkb = unit_nkb(p, un);
+    const int nkb = unit_nkb<kFma>(p, un);
     const uint32_t bytes = fma ? fma_stage_bytes(un.prec)
                                : xbytes + (bf16 ? (uint32_t)un.nbox * (kBoxRows * 128) : 0u);
     const int reserve_kb = max(0, nkb - (int)ns - 4);
@@ -817,6 +824,7 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h,
 // Streams the INT8/INT4 codes and fp16 scales of each quantised unit into the
 // staging ring, as far ahead as the ring allows, independently of the operand
 // stages (which wait on the tensor core); BF16 units are skipped.
+template <bool kFma>
 __device__ void code_producer(const Params& p, const Smem& s) {
   volatile int* abort_flag = s.abort_flag;
   const uint32_t nq = p.nq;
@@ -835,13 +843,13 @@ __device__ void code_producer(const Params& p, const Smem& s) {
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
     ++tseq;
-    if (un.prec == MOE_BF16 || unit_fma(un)) continue;
+    if (un.prec == MOE_BF16 || unit_fma<kFma>(un)) continue;
     const bool gu = unit_gu(un);
     const ExpertDesc* d = p.descs + un.e;
     const CUtensorMap* tw = gu ? &d->tm_w13 : &d->tm_w2;
     tmap_acquire(tw);
     prefetch_tmap(tw);
-    const int nkb = unit_nkb(p, un);
+    const int nkb = unit_nkb<kFma>(p, un);
     const bool int4 = un.prec == MOE_INT4;
     long long tr_wait = 0;
     (void)tr_wait;
@@ -901,7 +909,7 @@ __device__ __forceinline__ void mma_kblock_ts(uint32_t d, uint32_t a_tmem, uint6
   mma_bf16_ts(d, a_tmem + 24, b + 6, idesc, 1u);
 }
 
-template <bool kSwap>
+template <bool kSwap, bool kFma>
 __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
   const uint32_t acc_cols = p.acc_stride, a_tmem0 = tmem + p.a_col;
   volatile int* abort_flag = s.abort_flag;
@@ -924,8 +932,8 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
     mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
-    const int nkb = unit_nkb(p, un);
-    if (kSwap && unit_fma(un)) {  // computed and freed by the dequant warps
+    const int nkb = unit_nkb<kFma>(p, un);
+    if (kSwap && unit_fma<kFma>(un)) {  // computed and freed by the dequant warps
       for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
       ++tseq;
       continue;
@@ -1114,7 +1122,7 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
   const int lane = threadIdx.x & 31;
   const int c = ft & 15, rsub = ft >> 4;
   constexpr int kPairs = kInt4 ? 8 : 4;  // element pairs of a lane's chunk
-  const int nkb = unit_nkb(p, un);
+  const int nkb = unit_nkb<true>(p, un);
   float acc[8][N];
 #pragma unroll
   for (int j = 0; j < 8; ++j)
@@ -1281,6 +1289,7 @@ __device__ bool fma_dispatch(const Params& p, const Smem& s, const Unit& un, int
 // second half): INT4 slot = two k-blocks (half h -> k-block 2g + h, 32 code
 // bytes -> 64 elements -> 32 columns), INT8 slot = one k-block (half h ->
 // elements 32 h .. + 31 -> 16 columns).
+template <bool kFma>
 __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
   volatile int* abort_flag = s.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1319,8 +1328,8 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
     ++tseq;
-    const int nkb = unit_nkb(p, un);
-    if ((pub.flags & kUnitValid) && !unit_fma(un)) {
+    const int nkb = unit_nkb<kFma>(p, un);
+    if ((pub.flags & kUnitValid) && !unit_fma<kFma>(un)) {
       publish_rows(p, pub, lane);
       pub.flags = 0;
     }
@@ -1329,7 +1338,7 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
       continue;
     }
     if (tracer) FFN_TRACE_SET(tseq, kTrDqBeg, FFN_TRACE_NS());
-    if (unit_fma(un)) {
+    if (unit_fma<kFma>(un)) {
       long long tr[5] = {0, 0, 0, 0, 0};
       ok = un.prec == MOE_INT4
                ? fma_dispatch<true>(p, s, un, ft, st, sph, ffph, fdph, pub, tr)
@@ -1442,7 +1451,7 @@ __device__ void dequant(const Params& p, const Smem& s, int dtid) {
     if (lane == 0) mbar_arrive(&s.uempty[us]);
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
-    const int nkb = unit_nkb(p, un);
+    const int nkb = unit_nkb<false>(p, un);
     if (un.prec == MOE_BF16) {
       for (int kb = 0; kb < nkb; ++kb) advance(st, sph, ns);
       continue;
@@ -1528,7 +1537,7 @@ __device__ void dequant(const Params& p, const Smem& s, int dtid) {
 
 // ---------------------------------------------------------------- epilogue --
 
-template <bool kSwap>
+template <bool kSwap, bool kFma>
 __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
   const uint32_t acc_cols = p.acc_stride;
   volatile int* abort_flag = s.abort_flag;
@@ -1552,7 +1561,7 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
     advance(us, uph, kUR);
     if (!(un.flags & kUnitValid)) break;
     const bool gu = unit_gu(un);
-    if (kSwap && unit_fma(un)) {  // the dequant warps store and publish its rows
+    if (kSwap && unit_fma<kFma>(un)) {  // the dequant warps store and publish its rows
       ++tseq;
       continue;
     }
@@ -1661,7 +1670,7 @@ __device__ void epilogue(const Params& p, const Smem& s, uint32_t tmem) {
 }
 
 // ------------------------------------------------------------------ kernel --
-template <bool kSwap>
+template <bool kSwap, bool kFma>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_ffn_kernel(const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_h,
@@ -1719,18 +1728,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *s.tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) producer<kSwap>(&tm_x, &tm_h, &tm_xf, &tm_hf, p, s);
+    if (lane == 0) producer<kSwap, kFma>(&tm_x, &tm_h, &tm_xf, &tm_hf, p, s);
   } else if (warp == 1) {
-    if (lane == 0) mma_issuer<kSwap>(p, s, tmem);
+    if (lane == 0) mma_issuer<kSwap, kFma>(p, s, tmem);
   } else if (warp >= 4 && warp < 8) {
-    epilogue<kSwap>(p, s, tmem);
+    epilogue<kSwap, kFma>(p, s, tmem);
   } else if (warp == 14) {
-    if (lane == 0) code_producer(p, s);
+    if (lane == 0) code_producer<kFma>(p, s);
   } else if (warp == 15) {
-    if (lane == 0) scheduler<kSwap>(p, s);
+    if (lane == 0) scheduler<kSwap, kFma>(p, s);
   } else {
     if (kSwap) {
-      dequant_tmem(p, s, tmem);
+      dequant_tmem<kFma>(p, s, tmem);
     } else {
       const int dtid = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // warps 2, 3, 8 .. 13
       dequant(p, s, dtid);

@@ -409,7 +409,8 @@ int router_impl(const void* h, const void* w_router, int T, int H, int E, int k,
   const size_t smem = R::layout(npad, tm, ns, S).total;
   MOE_CHECK(smem <= R::kSmemLimit, MOE_ERR_UNSUPPORTED, "router tile does not fit (E=%d)", E);
   CUtensorMap tm_h, tm_w;
-  rc = encode_2d(&tm_h, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, H, tm, R::kKB,
+  const int hrows = std::min(tm, (T + 7) / 8 * 8);
+  rc = encode_2d(&tm_h, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, H, hrows, R::kKB,
                  CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != MOE_OK) return rc;
   rc = encode_2d(&tm_w, w_router, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, H, std::min(npad, 256),
@@ -424,6 +425,7 @@ int router_impl(const void* h, const void* w_router, int T, int H, int E, int k,
   prm.do_topk = do_topk;
   prm.npad = npad;
   prm.tm = tm;
+  prm.hrows = hrows;
   prm.nkb = nkb;
   prm.ns = ns;
   prm.logits = logits;
@@ -547,10 +549,13 @@ int set_ffn_attributes(int dev) {
   static std::atomic<bool> done[kMaxDevices];
   const bool cached = dev >= 0 && dev < kMaxDevices;
   if (cached && done[dev].load()) return MOE_OK;
-  MOE_CUDA_TRY(cudaFuncSetAttribute(moe::ffn::grouped_ffn_kernel<true>,
+  MOE_CUDA_TRY(cudaFuncSetAttribute(moe::ffn::grouped_ffn_kernel<true, true>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     moe::ffn::kSmemLimit));
-  MOE_CUDA_TRY(cudaFuncSetAttribute(moe::ffn::grouped_ffn_kernel<false>,
+  MOE_CUDA_TRY(cudaFuncSetAttribute(moe::ffn::grouped_ffn_kernel<true, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    moe::ffn::kSmemLimit));
+  MOE_CUDA_TRY(cudaFuncSetAttribute(moe::ffn::grouped_ffn_kernel<false, false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     moe::ffn::kSmemLimit));
   if (cached) done[dev].store(true);
@@ -613,6 +618,21 @@ int route_permute_gather_small(moe_layer_t L, const float* logits, const void* x
   return ok();
 }
 
+// Whether a launch of this layer can contain CUDA-core units: its shape allows
+// them and some expert's base precision (a forward sees that version or a BF16
+// one) spans at least kFmaMinStages stages in one of its projections.  Only
+// then does the launch take the kernel instance with the CUDA-core path.
+bool fma_possible(const moe_layer* L) {
+  if (!fma_capable(L->H, L->I)) return false;
+  for (int q : L->prec) {
+    if (q != MOE_INT8 && q != MOE_INT4) continue;
+    const int step = q == MOE_INT4 ? 256 : 128;
+    if (L->H / step >= moe::ffn::kFmaMinStages || L->I / step >= moe::ffn::kFmaMinStages)
+      return true;
+  }
+  return false;
+}
+
 // zero_counters = false: the caller has already zeroed the scheduler counters
 // on the stream (moe_layer_forward does so first, so that no memset node sits
 // between the layer's kernels).
@@ -665,7 +685,7 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
                  CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != MOE_OK) return rc;
   // CUDA-core units (swap mode): X rows of a tile in 128-element boxes, unswizzled
-  const int fma_rows = swap && fma_capable(L->H, L->I) ? kFmaRows : 0;
+  const int fma_rows = swap && fma_possible(L) ? kFmaRows : 0;
   memset(&tm_xf, 0, sizeof tm_xf);
   memset(&tm_hf, 0, sizeof tm_hf);
   if (fma_rows > 0) {
@@ -684,12 +704,15 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
 
   rc = set_ffn_attributes(dev);
   if (rc != MOE_OK) return rc;
-  if (swap)
-    MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<true>, dim3(grid), dim3(kThreads), smem, s, tm_x,
-                            tm_h, tm_xf, tm_hf, prm));
+  if (swap && fma_rows > 0)
+    MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<true, true>, dim3(grid), dim3(kThreads), smem, s,
+                            tm_x, tm_h, tm_xf, tm_hf, prm));
+  else if (swap)
+    MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<true, false>, dim3(grid), dim3(kThreads), smem, s,
+                            tm_x, tm_h, tm_xf, tm_hf, prm));
   else
-    MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<false>, dim3(grid), dim3(kThreads), smem, s, tm_x,
-                            tm_h, tm_xf, tm_hf, prm));
+    MOE_CUDA_TRY(launch_pdl(grouped_ffn_kernel<false, false>, dim3(grid), dim3(kThreads), smem,
+                            s, tm_x, tm_h, tm_xf, tm_hf, prm));
   return ok();
 }
 }  // namespace

@@ -24,7 +24,7 @@
 namespace moe {
 namespace router {
 
-constexpr int kThreads = 128;     // 4 warps; TMEM lane quadrant = warp
+constexpr int kThreads = 512;     // 16 warps; warp w reads TMEM lane quadrant w % 4
 constexpr int kKB = 64;           // K-elements per stage: one 128-byte swizzled row
 constexpr int kMaxE = 512;
 constexpr int kMaxCluster = 8;    // portable cluster size
@@ -36,6 +36,7 @@ struct Params {
   int T, H, E, k, renormalize, do_topk;
   int npad;   // E rounded up to 16
   int tm;     // token rows per tile
+  int hrows;  // rows per h copy: min(tm, T rounded up to 8); the MMA's other A rows are unused
   int nkb;    // H / kKB
   int ns;     // ring stages
   float* logits;       // [T][E] or null
@@ -115,8 +116,10 @@ __device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
 }
 
 // Grid (S, tiles), cluster (S, 1, 1).  Warp 0 lane 0 issues the TMA copies,
-// warp 1 lane 0 the MMAs; all four warps then read the accumulator (warp w
-// owns TMEM lanes 32w .. 32w + 31 = the tile's rows).  Every wait is bounded;
+// warp 1 lane 0 the MMAs; then all 16 warps drain the accumulator (warp w
+// reads TMEM lanes 32 (w % 4) .. + 31 = tile rows, every fourth 16-column
+// chunk), reduce and route: the top-k's dependent warp reductions need many
+// warps in flight.  Every wait is bounded;
 // a thread that gives up sets MOE_STATUS_WAIT_TIMEOUT and still takes part in
 // both cluster barriers, so no CTA waits for one that left.
 template <int KEYS>
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_h);
     prefetch_tmap(&tm_w);
     pdl_wait();  // h may come from the previous kernel in the stream
-    const uint32_t tx = (uint32_t)p.tm * 128u + (p.npad > 256 ? 2 * kWChunk : wstage_of(p.npad));
+    const uint32_t tx = (uint32_t)p.hrows * 128u + wstage_of(p.npad);
     int issued = 0;
     for (int i = 0; i < nkl; ++i) {
       const int st = i % p.ns;
@@ -219,10 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncwarp();
   const int pstride = p.npad + 4;
   float* part = reinterpret_cast<float*>(base);
-  const int r = warp * 32 + lane;
-  for (int c = 0; c < p.npad; c += 16) {
+  const int quad = warp & 3, r = quad * 32 + lane;
+  // the four warps of a lane quadrant take every fourth 16-column chunk
+  for (int c = (warp >> 2) * 16; c < p.npad; c += 64) {
     uint32_t v[16];
-    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c, v);
+    tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + c, v);
     tmem_ld_wait();
     if (ok && r < rows) {
       const uint32_t a = smem_u32(part + (size_t)r * pstride + c);
@@ -246,14 +250,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = threadIdx.x; i < (r_hi - r_lo) * c4n; i += kThreads) {
       const int rr = r_lo + i / c4n, c4 = i % c4n;
       const uint32_t off = part_s + ((uint32_t)rr * pstride + c4 * 4) * 4u;
-      float4 acc = ld_cluster_v4(mapa(off, 0));
-      for (int q = 1; q < S; ++q) {
-        const float4 v = ld_cluster_v4(mapa(off, (uint32_t)q));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
+      // all S remote loads in flight first, then the sum in rank order
+      float4 v[kMaxCluster];
+#pragma unroll
+      for (int q = 0; q < kMaxCluster; ++q)
+        if (q < S) v[q] = ld_cluster_v4(mapa(off, (uint32_t)q));
+      float4 acc = v[0];
+#pragma unroll
+      for (int q = 1; q < kMaxCluster; ++q)
+        if (q < S) {
+          acc.x += v[q].x;
+          acc.y += v[q].y;
+          acc.z += v[q].z;
+          acc.w += v[q].w;
+        }
       *reinterpret_cast<float4*>(zbuf + (size_t)(rr - r_lo) * p.npad + c4 * 4) = acc;
     }
   }
