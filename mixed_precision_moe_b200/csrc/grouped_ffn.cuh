@@ -602,9 +602,11 @@ __device__ void scheduler(const Params& p, const Smem& s) {
       gph ^= 1u;
     }
     int u;
-    if (!kSwap) {
-      // tile mode: every gate/up unit, then every down unit, in order; the first
-      // unit of CTA b is unit b, later ones come from the counter
+    if (!kSwap || !kFma) {
+      // every gate/up unit, then every down unit, in order; the first unit of
+      // CTA b is unit b, later ones come from the counter.  Without CUDA-core
+      // units the gate/up units of an expert finish close together and this
+      // order was measured 0.7 % faster at decode than the ready list below.
       u = first ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.counter, 1);
     } else if (first && (int)blockIdx.x < total_gu) {
       u = blockIdx.x;

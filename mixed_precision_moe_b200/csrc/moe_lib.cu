@@ -358,17 +358,44 @@ int router_check(const void* h, const void* w_router, int T, int H, int E, int k
   return MOE_OK;
 }
 
+// Attributes of router_topk_kernel<KEYS> on the current device, set once: the
+// shared-memory limit and clusters of up to 16 CTAs (non-portable).  Returns
+// the largest cluster size to use: 16 if a cluster of 16 CTAs with the full
+// shared memory fits on this GPU, else 8.
+template <int KEYS>
+int router_attributes(int dev) {
+  static std::atomic<int> max_cluster[kMaxDevices];
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && max_cluster[dev].load() != 0) return max_cluster[dev].load();
+  auto kern = moe::router::router_topk_kernel<KEYS>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)moe::router::kSmemLimit) != cudaSuccess)
+    return 0;
+  int m = 8;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16);
+    cfg.blockDim = dim3(moe::router::kThreads);
+    cfg.dynamicSmemBytes = moe::router::kSmemLimit;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1) m = 16;
+  }
+  cudaGetLastError();  // a refused attribute or query leaves no sticky error
+  if (cached) max_cluster[dev].store(m);
+  return m;
+}
+
 template <int KEYS>
 int router_launch(const CUtensorMap& tm_h, const CUtensorMap& tm_w, const moe::router::Params& prm,
-                  int S, int tiles, size_t smem, int dev, cudaStream_t s) {
-  static std::atomic<bool> done[kMaxDevices];
-  const bool cached = dev >= 0 && dev < kMaxDevices;
-  if (!(cached && done[dev].load())) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(moe::router::router_topk_kernel<KEYS>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)moe::router::kSmemLimit));
-    if (cached) done[dev].store(true);
-  }
+                  int S, int tiles, size_t smem, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S, tiles);
   cfg.blockDim = dim3(moe::router::kThreads);
@@ -388,7 +415,8 @@ int router_launch(const CUtensorMap& tm_h, const CUtensorMap& tm_w, const moe::r
 }
 
 // z = W_r h on the tensor cores, then (do_topk) the top-k of every token.
-// Cluster size S: the largest power of two <= 8 (and <= H / 64) that keeps
+// Cluster size S: the largest power of two <= 16 (8 where a 16-CTA cluster
+// does not fit; and <= H / 64) that keeps
 // tiles * S within the SM count; stages: as many as the shared memory holds,
 // up to the k-blocks of one CTA.
 int router_impl(const void* h, const void* w_router, int T, int H, int E, int k, int renormalize,
@@ -401,8 +429,15 @@ int router_impl(const void* h, const void* w_router, int T, int H, int E, int k,
   const int npad = R::npad_of(E), tm = R::tm_of(E), nkb = H / R::kKB;
   const int tiles = (T + tm - 1) / tm;
   const int nsm = std::max(1, num_sms(dev));
+  const int keys = (E + 31) / 32;
+  const int max_cluster = keys <= 1   ? router_attributes<1>(dev)
+                          : keys <= 2 ? router_attributes<2>(dev)
+                          : keys <= 4 ? router_attributes<4>(dev)
+                          : keys <= 8 ? router_attributes<8>(dev)
+                                      : router_attributes<16>(dev);
+  MOE_CHECK(max_cluster > 0, MOE_ERR_CUDA, "cannot set the router kernel's attributes");
   int S = 1;
-  while (S * 2 <= R::kMaxCluster && S * 2 <= nkb && tiles * S * 2 <= nsm) S *= 2;
+  while (S * 2 <= max_cluster && S * 2 <= nkb && tiles * S * 2 <= nsm) S *= 2;
   const int nkl_max = (nkb + S - 1) / S;
   int ns = 1;
   while (ns < nkl_max && R::layout(npad, tm, ns + 1, S).total <= R::kSmemLimit) ++ns;
@@ -431,13 +466,12 @@ int router_impl(const void* h, const void* w_router, int T, int H, int E, int k,
   prm.logits = logits;
   prm.topk_idx = topk_idx;
   prm.topk_w = topk_w;
-  const int keys = (E + 31) / 32;
   cudaStream_t s = as_stream(stream);
-  rc = keys <= 1   ? router_launch<1>(tm_h, tm_w, prm, S, tiles, smem, dev, s)
-       : keys <= 2 ? router_launch<2>(tm_h, tm_w, prm, S, tiles, smem, dev, s)
-       : keys <= 4 ? router_launch<4>(tm_h, tm_w, prm, S, tiles, smem, dev, s)
-       : keys <= 8 ? router_launch<8>(tm_h, tm_w, prm, S, tiles, smem, dev, s)
-                   : router_launch<16>(tm_h, tm_w, prm, S, tiles, smem, dev, s);
+  rc = keys <= 1   ? router_launch<1>(tm_h, tm_w, prm, S, tiles, smem, s)
+       : keys <= 2 ? router_launch<2>(tm_h, tm_w, prm, S, tiles, smem, s)
+       : keys <= 4 ? router_launch<4>(tm_h, tm_w, prm, S, tiles, smem, s)
+       : keys <= 8 ? router_launch<8>(tm_h, tm_w, prm, S, tiles, smem, s)
+                   : router_launch<16>(tm_h, tm_w, prm, S, tiles, smem, s);
   return rc;
 }
 }  // namespace

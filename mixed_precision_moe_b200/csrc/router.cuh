@@ -27,7 +27,7 @@ namespace router {
 constexpr int kThreads = 512;     // 16 warps; warp w reads TMEM lane quadrant w % 4
 constexpr int kKB = 64;           // K-elements per stage: one 128-byte swizzled row
 constexpr int kMaxE = 512;
-constexpr int kMaxCluster = 8;    // portable cluster size
+constexpr int kMaxCluster = 16;   // non-portable cluster size (8 is portable)
 constexpr uint32_t kHStage = 16384;   // 128 rows x 128 B (M = 128 reads all of it)
 constexpr uint32_t kWChunk = 32768;   // 256 expert rows x 128 B
 constexpr size_t kSmemLimit = 227 * 1024;
@@ -115,7 +115,7 @@ __device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
   return v;
 }
 
-// Grid (S, tiles), cluster (S, 1, 1).  Warp 0 lane 0 issues the TMA copies,
+// Grid (S, tiles), cluster (S, 1, 1), S <= 16.  Warp 0 lane 0 issues the TMA copies,
 // warp 1 lane 0 the MMAs; then all 16 warps drain the accumulator (warp w
 // reads TMEM lanes 32 (w % 4) .. + 31 = tile rows, every fourth 16-column
 // chunk), reduce and route: the top-k's dependent warp reductions need many
@@ -145,6 +145,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb0 = s * p.nkb / S, nkl = (s + 1) * p.nkb / S - kb0;
   const int nchunk = p.npad > 256 ? 2 : 1;
 
+  // Thread 0 initialises the barriers and, as the producer, issues the copies
+  // of the first ns stages at once (they need no free stage), overlapping the
+  // TMEM allocation and the block-wide sync that publishes it.
+  const uint32_t tx = (uint32_t)p.hrows * 128u + wstage_of(p.npad);
+  auto issue = [&](int i) {
+    const int st = i % p.ns;
+    uint8_t* hs = base + st * stage;
+    uint8_t* ws = hs + kHStage;
+    const int kx = (kb0 + i) * kKB;
+    mbar_arrive_expect_tx(&full[st], tx);
+    tma_load_2d(hs, &tm_h, kx, row0, &full[st]);
+    for (int c = 0; c < nchunk; ++c) tma_load_2d(ws + c * kWChunk, &tm_w, kx, c * 256, &full[st]);
+  };
+  const int first = min(nkl, p.ns);
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.ns; ++i) {
       mbar_init(&full[i], 1);
@@ -153,6 +167,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    prefetch_tmap(&tm_h);
+    prefetch_tmap(&tm_w);
+    pdl_wait();  // h may come from the previous kernel in the stream
+    for (int i = 0; i < first; ++i) issue(i);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, ncols);
@@ -165,24 +183,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    prefetch_tmap(&tm_h);
-    prefetch_tmap(&tm_w);
-    pdl_wait();  // h may come from the previous kernel in the stream
-    const uint32_t tx = (uint32_t)p.hrows * 128u + wstage_of(p.npad);
-    int issued = 0;
-    for (int i = 0; i < nkl; ++i) {
+    // ------------------------------------- producer: the stages beyond ns
+    int issued = first;
+    for (int i = first; i < nkl; ++i) {
       const int st = i % p.ns;
-      if (i >= p.ns && !mbar_wait(&empty[st], ((i / p.ns) - 1) & 1, abort_flag)) {
+      if (!mbar_wait(&empty[st], ((i / p.ns) - 1) & 1, abort_flag)) {
         *abort_flag = 1;
         break;
       }
-      uint8_t* hs = base + st * stage;
-      uint8_t* ws = hs + kHStage;
-      const int kx = (kb0 + i) * kKB;
-      mbar_arrive_expect_tx(&full[st], tx);
-      tma_load_2d(hs, &tm_h, kx, row0, &full[st]);
-      for (int c = 0; c < nchunk; ++c) tma_load_2d(ws + c * kWChunk, &tm_w, kx, c * 256, &full[st]);
+      issue(i);
       issued = i + 1;
     }
     if (*abort_flag) {  // let the copies in flight land before the bytes are reused
@@ -267,9 +276,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<float4*>(zbuf + (size_t)(rr - r_lo) * p.npad + c4 * 4) = acc;
     }
   }
-  cluster_sync();  // no CTA reads a peer's shared memory after this point
+  __syncthreads();  // this CTA's reduced rows are complete
 
   // ----------------------------------------------- logits and the top-k
+  // (before the exit barrier below: they read only this CTA's own rows, while
+  // peers may still be reading its partials)
   auto zrow = [&](int rr) -> const float* {
     return S > 1 ? zbuf + (size_t)(rr - r_lo) * p.npad : part + (size_t)rr * pstride;
   };
@@ -291,6 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.topk_w[t * p.k + lane] = w;
       }
     }
+  __syncwarp();
+  cluster_sync();  // no CTA leaves while a peer may still read its partials
 }
 
 }  // namespace router

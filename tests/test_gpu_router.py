@@ -8,10 +8,10 @@ oracle computes z in binary64 from the same bf16 bits.
 
 Tolerance of the logits, from the arithmetic: every bf16 x bf16 product is
 exact in fp32, and the kernel sums them in fp32 on the tensor cores (four K=16
-MMAs per 64-element k-block, then at most 8 partial sums of the cluster's K
+MMAs per 64-element k-block, then at most 16 partial sums of the cluster's K
 split).  Counting two units of 2^-23 (relative to the sum of the products'
 magnitudes) per MMA and one per partial sum gives
-    |z_gpu - z| <= delta = (8 * H/64 + 8 + 2) * 2^-23 * sum_h |h_h W_eh|.
+    |z_gpu - z| <= delta = (8 * H/64 + 16 + 2) * 2^-23 * sum_h |h_h W_eh|.
 The top-k is an integer decision made in fp32 on the kernel's logits, so the
 exact ids are compared where the oracle's logits decide them by more than the
 tolerance, and elsewhere the selection must be a valid top-k of some logits
@@ -46,7 +46,7 @@ def _delta(h_bits, w_bits):
     H = h_bits.shape[1]
     a = np.abs(synth.bf16_bits_to_f32(h_bits).astype(np.float64))
     b = np.abs(synth.bf16_bits_to_f32(w_bits).astype(np.float64))
-    return (8 * (H // 64) + 10) * 2.0 ** -23 * (a @ b.T)
+    return (8 * (H // 64) + 18) * 2.0 ** -23 * (a @ b.T)
 
 
 def _check_topk_valid(idx, w, zo, delta, k, renorm):
@@ -119,7 +119,8 @@ def test_router_topk_against_oracle(name, T, H, E, k, zipf_s, renorm):
     assert np.all(err <= delta), f"{name}: logit error {err.max():.3e} (ratio {np.max(err / delta):.3f})"
     decided = _check_topk_valid(idx.cpu().numpy(), w.cpu().numpy().astype(np.float64), zo, delta,
                                 k, renorm)
-    assert decided >= 0.9 * T, f"{name}: only {decided} of {T} tokens decided by the oracle"
+    # not vacuous: most tokens are decided by the oracle alone (>= 0.906 on every case here)
+    assert decided >= 0.85 * T, f"{name}: only {decided} of {T} tokens decided by the oracle"
 
     # the fused top-k equals the separate routing kernel on the kernel's own logits
     idx2, w2 = B.moe_route_topk(logits, k, renorm)
