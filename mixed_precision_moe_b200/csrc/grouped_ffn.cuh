@@ -91,12 +91,14 @@ struct alignas(64) ExpertDesc {
   CUtensorMap tm_q2f;   // INT8/INT4 codes of W2; box 128 rows x 128 B
   CUtensorMap tm_s13f;  // INT8/INT4 scales [H/128][2I] as [G][2][I]; box (INT4: 2, INT8: 1) x 2 x 64
   CUtensorMap tm_s2f;   // INT8/INT4 scales [I/128][H]; box (2 | 1) groups x 128 rows
+  CUtensorMap tm_q2h;   // INT8/INT4 codes of W2; box 64 rows x 128 B (half-height down units)
+  CUtensorMap tm_s2h;   // INT8/INT4 scales [I/128][H]; box (2 | 1) groups x 64 rows
   const __half* s13;    // [H/128][2I]
   const __half* s2;     // [I/128][H]
   int prec;             // MOE_BF16 / MOE_INT8 / MOE_INT4, -1 when unset
   int pad[11];
 };
-static_assert(sizeof(ExpertDesc) == 832, "descriptor layout");
+static_assert(sizeof(ExpertDesc) == 1088, "descriptor layout");
 
 struct Unit {
   int e, prec, wrow0, nbox;  // expert, precision, first weight row (of each half), 128-row boxes
@@ -330,6 +332,21 @@ __device__ __forceinline__ int tiles_of(int n, const Params& p) {
   return n > 0 ? (n + p.xrows - 1) / p.xrows : 0;
 }
 
+// CUDA-core down units of an expert (INT8/INT4, at most fma_rows rows, I of at
+// least kFmaMinStages stages) are 64 weight rows high, twice as many as the
+// 128-row units of the tensor-core path: at one or two tokens per expert a
+// down unit streams a long K, and halving it keeps more SMs busy at the end.
+template <bool kSwap, bool kFma>
+__device__ __forceinline__ bool fma_down(const Params& p, int prec, int nrows) {
+  if (!kFma || !kSwap || prec == MOE_BF16 || nrows > p.fma_rows) return false;
+  return p.I / (prec == MOE_INT4 ? 256 : 128) >= kFmaMinStages;
+}
+
+template <bool kSwap, bool kFma>
+__device__ __forceinline__ int down_units_of(const Params& p, int prec, int nrows) {
+  return tiles_of(nrows, p) * p.nwb_dn * (fma_down<kSwap, kFma>(p, prec, nrows) ? 2 : 1);
+}
+
 // The unit table, built by every CTA from expert_offsets and the precision
 // array: the experts with rows, with their first unit index; unit indices =
 // every gate/up unit, then every down unit, experts in the same order:
@@ -347,14 +364,14 @@ __device__ __forceinline__ int tiles_of(int n, const Params& p) {
 // my_prec: p.prec[threadIdx.x] (read by the caller before griddepcontrol.wait:
 // the precisions are written only by write_desc_kernel, which never lets a
 // dependent launch start before it completes).
-template <bool kSwap>
+template <bool kSwap, bool kFma>
 __device__ void build_entries(const Params& p, const Smem& s, int my_prec) {
   static_assert(kThreads >= kMaxE, "one thread per expert");
   constexpr int kWarps = kThreads / 32;
   constexpr int kC = kSwap ? 1 : 3;            // classes in unit order
-  int* wsum = reinterpret_cast<int*>(s.q_st);  // [kWarps][2 kC]; staging is free until the mainloop
+  int* wsum = reinterpret_cast<int*>(s.q_st);  // [kWarps][3 kC]; staging is free until the mainloop
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int off = 0, n = 0, prec = -1, cls = -1, tiles = 0;
+  int off = 0, n = 0, prec = -1, cls = -1, tiles = 0, dnu = 0;
   if (tid < p.E) {
     off = p.offsets[tid];
     n = p.offsets[tid + 1] - off;
@@ -369,63 +386,69 @@ __device__ void build_entries(const Params& p, const Smem& s, int my_prec) {
       if (prec == MOE_INT4 || prec == MOE_INT8 || prec == MOE_BF16) {
         cls = kSwap ? 0 : (prec == MOE_INT4 ? 0 : prec == MOE_INT8 ? 1 : 2);
         tiles = tiles_of(n, p);
+        dnu = down_units_of<kSwap, kFma>(p, prec, n);
       } else {
         flag_status(MOE_STATUS_UNSET_EXPERT);
       }
     }
   }
-  // inclusive warp scans of v[c] = tiles and v[kC + c] = entries of class c
-  int v[2 * kC], incl[2 * kC];
+  // inclusive warp scans of v[c] = tiles, v[kC + c] = entries and v[2 kC + c]
+  // = down units of class c
+  int v[3 * kC], incl[3 * kC];
 #pragma unroll
   for (int c = 0; c < kC; ++c) {
     v[c] = cls == c ? tiles : 0;
     v[kC + c] = cls == c ? 1 : 0;
+    v[2 * kC + c] = cls == c ? dnu : 0;
   }
 #pragma unroll
-  for (int i = 0; i < 2 * kC; ++i) {
+  for (int i = 0; i < 3 * kC; ++i) {
     incl[i] = v[i];
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       const int x = __shfl_up_sync(0xffffffffu, incl[i], d);
       if (lane >= d) incl[i] += x;
     }
-    if (lane == 31) wsum[warp * 2 * kC + i] = incl[i];
+    if (lane == 31) wsum[warp * 3 * kC + i] = incl[i];
   }
   __syncthreads();
-  int before[2 * kC], total[2 * kC];  // sums over earlier warps / over all warps
+  int before[3 * kC], total[3 * kC];  // sums over earlier warps / over all warps
 #pragma unroll
-  for (int i = 0; i < 2 * kC; ++i) before[i] = total[i] = 0;
+  for (int i = 0; i < 3 * kC; ++i) before[i] = total[i] = 0;
   for (int w = 0; w < kWarps; ++w)
 #pragma unroll
-    for (int i = 0; i < 2 * kC; ++i) {
-      const int x = wsum[w * 2 * kC + i];
+    for (int i = 0; i < 3 * kC; ++i) {
+      const int x = wsum[w * 3 * kC + i];
       total[i] += x;
       if (w < warp) before[i] += x;
     }
-  int total_tiles = 0, total_ents = 0;
+  int total_tiles = 0, total_ents = 0, total_dn = 0;
 #pragma unroll
   for (int c = 0; c < kC; ++c) {
     total_tiles += total[c];
     total_ents += total[kC + c];
+    total_dn += total[2 * kC + c];
   }
   const int total_gu = total_tiles * p.nwb_gu;
 #pragma unroll
   for (int c = 0; c < kC; ++c) {
     if (cls != c) continue;
-    int tile_base = 0, ent_base = 0;
+    int tile_base = 0, ent_base = 0, dn_base = 0;
 #pragma unroll
     for (int c2 = 0; c2 < c; ++c2) {
       tile_base += total[c2];
       ent_base += total[kC + c2];
+      dn_base += total[2 * kC + c2];
     }
     const int t = tile_base + before[c] + incl[c] - v[c];  // token tiles before this expert
     const int en = ent_base + before[kC + c] + incl[kC + c] - v[kC + c];
+    const int dn = dn_base + before[2 * kC + c] + incl[2 * kC + c] - v[2 * kC + c];
     s.entries[en] = Entry{t * p.nwb_gu, tid | (prec << 16), off, n};
-    s.ub_dn[en] = total_gu + t * p.nwb_dn;
+    s.ub_dn[en] = total_gu + dn;
   }
   if (tid == 0) {
     *s.n_units_gu = total_gu;
-    *s.n_units = total_gu + total_tiles * p.nwb_dn;
+    *s.n_units = total_gu + total_dn;
     *s.n_entries = total_ents;
   }
 }
@@ -442,7 +465,8 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
       hi = mid - 1;
   }
   const Entry en = s.entries[lo];
-  const int nwb = gu ? p.nwb_gu : p.nwb_dn;
+  const bool half = !gu && fma_down<kSwap, kFma>(p, en.e_prec >> 16, en.nrows);
+  const int nwb = gu ? p.nwb_gu : p.nwb_dn * (half ? 2 : 1);
   const int local = u - (gu ? en.unit_begin : s.ub_dn[lo]);
   const int tt = local / nwb, wb = local % nwb;
   Unit un;
@@ -454,8 +478,8 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, const Smem& s, int 
     un.wrow0 = wb * (kSwap ? 64 : 128);
     un.nbox = kSwap ? 1 : 2;
   } else {
-    un.wrow0 = wb * (kSwap ? 128 : 256);
-    un.nbox = min(kSwap ? 1 : 2, (p.H - un.wrow0) / kBoxRows);
+    un.wrow0 = wb * (kSwap ? (half ? kBoxRows / 2 : kBoxRows) : 256);
+    un.nbox = half ? 1 : min(kSwap ? 1 : 2, (p.H - un.wrow0) / kBoxRows);
   }
   // CUDA-core units: an INT8/INT4 expert with at most fma_rows rows runs a
   // projection on CUDA cores when its K spans at least kFmaMinStages stages.
@@ -527,9 +551,10 @@ __device__ __forceinline__ int unit_nkb(const Params& p, const Unit& un) {
 }
 
 // Bytes a CUDA-core stage receives: codes, X (one or two 128-K boxes) and scales.
-__device__ __forceinline__ uint32_t fma_stage_bytes(int prec) {
+// rows: the unit's weight rows (128; 64 for a CUDA-core down unit).
+__device__ __forceinline__ uint32_t fma_stage_bytes(int prec, uint32_t rows) {
   const uint32_t boxes = prec == MOE_INT4 ? 2u : 1u;
-  return kBoxRows * 128 + boxes * (kFmaRows * 256 + kBoxRows * 2);
+  return rows * 128 + boxes * (kFmaRows * 256 + rows * 2);
 }
 
 __device__ __forceinline__ int ld_acquire(const int* ptr) {
@@ -651,7 +676,8 @@ __device__ void scheduler(const Params& p, const Smem& s) {
         const int v = ld_acquire(p.ready + scan_slot);
         if (v != 0) {
           const int ent = v - 1;
-          const int nd = p.nwb_dn * tiles_of(s.entries[ent].nrows, p);
+          const int nd = down_units_of<kSwap, kFma>(p, s.entries[ent].e_prec >> 16,
+                                                    s.entries[ent].nrows);
           if (dn_j < scan_cum + nd) {
             u = s.ub_dn[ent] + (dn_j - scan_cum);
             dn_j = -1;
@@ -674,7 +700,7 @@ __device__ void scheduler(const Params& p, const Smem& s) {
       un = decode_unit<kSwap, kFma>(p, s, u);
       const ExpertDesc* d = p.descs + un.e;
       if (unit_fma<kFma>(un))
-        prefetch_tmap(unit_gu(un) ? &d->tm_q13f : &d->tm_q2f);
+        prefetch_tmap(unit_gu(un) ? &d->tm_q13f : &d->tm_q2h);
       else
         prefetch_tmap(unit_gu(un) ? &d->tm_w13 : &d->tm_w2);
       if (!unit_gu(un) && !wait_gate_up(p, un, abort_flag)) {
@@ -738,15 +764,16 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h,
     const bool fma = kSwap && unit_fma<kFma>(un);
     const bool int4 = un.prec == MOE_INT4;
     const ExpertDesc* d = p.descs + un.e;
-    const CUtensorMap* tw = fma ? (gu ? &d->tm_q13f : &d->tm_q2f) : (gu ? &d->tm_w13 : &d->tm_w2);
-    const CUtensorMap* tsc = gu ? &d->tm_s13f : &d->tm_s2f;
+    // (CUDA-core down units are 64 rows high: the half-height maps)
+    const CUtensorMap* tw = fma ? (gu ? &d->tm_q13f : &d->tm_q2h) : (gu ? &d->tm_w13 : &d->tm_w2);
+    const CUtensorMap* tsc = gu ? &d->tm_s13f : &d->tm_s2h;
     const CUtensorMap* tx = fma ? (gu ? tm_xf : tm_hf) : (gu ? tm_x : tm_h);
     const bool bf16 = un.prec == MOE_BF16;
     if (bf16 || fma) tmap_acquire(tw);
     if (fma) tmap_acquire(tsc);
     if (!gu) fence_proxy_async_global();  // h rows published (scheduler's acquire) -> TMA reads
     const int nkb = unit_nkb<kFma>(p, un);
-    const uint32_t bytes = fma ? fma_stage_bytes(un.prec)
+    const uint32_t bytes = fma ? fma_stage_bytes(un.prec, gu ? kBoxRows : kBoxRows / 2)
                                : xbytes + (bf16 ? (uint32_t)un.nbox * (kBoxRows * 128) : 0u);
     const int reserve_kb = max(0, nkb - (int)ns - 4);
     long long tr_wait = 0;
@@ -1107,7 +1134,7 @@ __device__ __forceinline__ uint32_t nib_f32(uint32_t a, uint32_t b) {
   return d;
 }
 
-template <int N, bool kInt4>
+template <int N, bool kInt4, bool kHalf>
 __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const Unit& un, int ft,
                                          uint32_t& st, uint32_t& sph, uint32_t& ffph,
                                          uint32_t& fdph, Unit& pub, long long* tr) {
@@ -1125,6 +1152,7 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
   const int c = ft & 15, rsub = ft >> 4;
   constexpr int kPairs = kInt4 ? 8 : 4;  // element pairs of a lane's chunk
   const int nkb = unit_nkb<true>(p, un);
+  constexpr int kJ = kHalf ? 4 : 8;  // rows 16 j + rsub of the unit (128, or 64 for kHalf)
   float acc[8][N];
 #pragma unroll
   for (int j = 0; j < 8; ++j)
@@ -1168,9 +1196,10 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
         sx[n] = 0.0f;
       }
     }
-    const __half* sc = reinterpret_cast<const __half*>(xs + kFmaXBytes) + (kInt4 ? (c >> 3) * 128 : 0);
+    const __half* sc = reinterpret_cast<const __half*>(xs + kFmaXBytes) +
+                       (kInt4 ? (c >> 3) * (kHalf ? kBoxRows / 2 : kBoxRows) : 0);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kJ; ++j) {
       const int r = 16 * j + rsub;
       const uint2 w = *reinterpret_cast<const uint2*>(codes + r * 128 + c * 8);
       const float sr = __half2float(sc[r]);
@@ -1231,7 +1260,7 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
   const long long c3 = FFN_CLOCK();
   // sum the 16 lanes (K-chunks) of each row; every lane ends with the totals
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
+  for (int j = 0; j < kJ; ++j)
 #pragma unroll
     for (int n = 0; n < N; ++n) {
       float v = acc[j][n];
@@ -1252,7 +1281,7 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
     pub = un;  // published later (deferred publication)
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < kJ; ++j)
 #pragma unroll
       for (int n = 0; n < N; ++n)
         if (c == n && n < un.nrows)
@@ -1267,14 +1296,15 @@ template <bool kInt4>
 __device__ bool fma_dispatch(const Params& p, const Smem& s, const Unit& un, int ft, uint32_t& st,
                              uint32_t& sph, uint32_t& ffph, uint32_t& fdph, Unit& pub,
                              long long* tr) {
-  static_assert(kFmaRows >= 1 && kFmaRows <= 4, "CUDA-core tiles of 1 to 4 rows");
-  if (kFmaRows >= 4 && un.nrows == 4)
-    return fma_unit<4, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
-  if (kFmaRows >= 3 && un.nrows == 3)
-    return fma_unit<3, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+  static_assert(kFmaRows >= 1 && kFmaRows <= 2, "CUDA-core tiles of 1 or 2 rows");
+  if (!unit_gu(un)) {  // down units: 64 weight rows
+    if (kFmaRows >= 2 && un.nrows == 2)
+      return fma_unit<2, kInt4, true>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+    return fma_unit<1, kInt4, true>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+  }
   if (kFmaRows >= 2 && un.nrows == 2)
-    return fma_unit<2, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
-  return fma_unit<1, kInt4>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+    return fma_unit<2, kInt4, false>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+  return fma_unit<1, kInt4, false>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
 }
 
 // One staging slot holds an INT4 group (128 K-elements = two k-blocks) or an
@@ -1722,7 +1752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   FFN_KSTAMP(1);
   pdl_wait();           // inputs of the previous kernels are complete from here on
-  build_entries<kSwap>(p, s, my_prec);  // contains a __syncthreads
+  build_entries<kSwap, kFma>(p, s, my_prec);  // contains a __syncthreads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

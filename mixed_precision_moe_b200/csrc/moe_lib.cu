@@ -144,7 +144,12 @@ int encode_weights(moe::ffn::ExpertDesc* d, const moe_expert_weights* w, int pre
   rc = encode_3d(&d->tm_s13f, w->s13, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, H / 128, 2, I, gs, 2, 64,
                  none);
   if (rc != MOE_OK) return rc;
-  return encode_2d(&d->tm_s2f, w->s2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, I / 128, H, gs, 128,
+  rc = encode_2d(&d->tm_s2f, w->s2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, I / 128, H, gs, 128, none);
+  if (rc != MOE_OK) return rc;
+  // half-height down units (64 rows) of the CUDA-core path
+  rc = encode_2d(&d->tm_q2h, w->w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H, cols2, 64, 128, none);
+  if (rc != MOE_OK) return rc;
+  return encode_2d(&d->tm_s2h, w->s2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, I / 128, H, gs, 64,
                    none);
 }
 
