@@ -25,9 +25,9 @@
 //                into a staging ring, running ahead of the operand stages.
 //   warp 1       TMEM owner + MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16
 //                -> fp32) into double-buffered TMEM accumulators.
-//   warps 2,3,8-13  dequant: staged codes x scale -> bf16, into shared memory
-//                (tile mode) or straight into TMEM as the MMA's A operand
-//                (swap mode).
+//   warps 2,3,8-13  dequant: staged codes x scale -> bf16, into the shared-
+//                memory weight stage (the MMA's B operand in tile mode, its A
+//                operand in swap mode).
 //   warps 4-7    epilogue: tcgen05.ld, SwiGLU or copy, bf16 stores; gate/up
 //                epilogues publish their rows with a release counter.
 // A work unit is (projection, expert, block of weight rows, tile of rows of
@@ -134,7 +134,6 @@ struct Params {
   int xrows;               // rows of an X stage = rows of a token tile (multiple of 16, <= 128)
   int ns, nq;              // ring depths
   int acc_stride;          // TMEM columns per accumulator buffer
-  int a_col;               // swap mode: TMEM column of the first A stage (32 columns each)
   int fma_rows;            // swap mode: INT8/INT4 experts with <= fma_rows rows run on CUDA cores
 };
 
@@ -913,8 +912,10 @@ __device__ void code_producer(const Params& p, const Smem& s) {
 // -------------------------------------------------------------- MMA issuer --
 // TMEM columns: tile mode uses two 256-column accumulators; swap mode uses two
 // accumulators of acc_stride columns (the power of two >= the token tile, so
-// N <= acc_stride) and, from column a_col = 2 * acc_stride, one 32-column A
-// stage per operand stage (64 K-elements x 128 rows of dequantised weights).
+// N <= acc_stride).  Every MMA reads both operands from shared memory: in swap
+// mode the dequantised INT8/INT4 weights are written into the weight stage in
+// the layout a BF16 box arrives in (measured 1 % faster for the decode FFN
+// than A operands in TMEM, whose MMA form issued ~1.5x slower per stage).
 
 // Four K=16 MMAs over one 64-element k-block.  The operand descriptors are
 // formed once per stage by adding to base descriptors (the start-address field
@@ -930,17 +931,9 @@ __device__ __forceinline__ void mma_kblock_ss(uint32_t d, uint64_t a, uint64_t b
   mma_bf16_ss(d, a + 6, b + 6, idesc, 1u);
 }
 
-__device__ __forceinline__ void mma_kblock_ts(uint32_t d, uint32_t a_tmem, uint64_t b,
-                                              uint32_t idesc, uint32_t acc0) {
-  mma_bf16_ts(d, a_tmem, b, idesc, acc0);
-  mma_bf16_ts(d, a_tmem + 8, b + 2, idesc, 1u);
-  mma_bf16_ts(d, a_tmem + 16, b + 4, idesc, 1u);
-  mma_bf16_ts(d, a_tmem + 24, b + 6, idesc, 1u);
-}
-
 template <bool kSwap, bool kFma>
 __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
-  const uint32_t acc_cols = p.acc_stride, a_tmem0 = tmem + p.a_col;
+  const uint32_t acc_cols = p.acc_stride;
   volatile int* abort_flag = s.abort_flag;
   const uint32_t ns = p.ns;
   const uint64_t wdesc0 = smem_desc_sw128(smem_u32(s.w_st));
@@ -976,8 +969,6 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
     const uint32_t d_tmem = tmem + abuf * acc_cols;
     const int n = kSwap ? max(16, (un.nrows + 15) & ~15) : un.nbox * kBoxRows;
     const uint32_t idesc = idesc_bf16_f32(128, n);
-    const bool quant = un.prec != MOE_BF16;
-    const bool a_in_tmem = kSwap && quant;  // dequantised weights live in TMEM
     long long tr_wait = 0, tr_issue = 0;
     (void)tr_wait;
     (void)tr_issue;
@@ -993,9 +984,7 @@ __device__ void mma_issuer(const Params& p, const Smem& s, uint32_t tmem) {
       tc_fence_after();
       const uint64_t xd = xdesc0 + st * xstep, wd = wdesc0 + st * wstep;
       const uint32_t acc0 = kb != 0;
-      if (a_in_tmem)
-        mma_kblock_ts(d_tmem, a_tmem0 + st * 32, xd, idesc, acc0);
-      else if (kSwap)
+      if (kSwap)
         mma_kblock_ss(d_tmem, wd, xd, idesc, acc0);
       else
         mma_kblock_ss(d_tmem, xd, wd, idesc, acc0);
@@ -1315,20 +1304,20 @@ __device__ bool fma_dispatch(const Params& p, const Smem& s, const Unit& un, int
 // (chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)).  Each warp signals
 // its own part (barrier counts are kDequantWarps), so the warps never wait on
 // one another.
-// Swap mode: dequantised weights go to TMEM instead of shared memory.  Warp w
-// owns TMEM lane quarter w % 4 (= weight rows 32 (w % 4) .. + 31 of the unit,
-// one row per thread) and one half of each staging slot (warps 10..13 the
-// second half): INT4 slot = two k-blocks (half h -> k-block 2g + h, 32 code
-// bytes -> 64 elements -> 32 columns), INT8 slot = one k-block (half h ->
-// elements 32 h .. + 31 -> 16 columns).
+// Swap mode: dequantised weights go into the stage's weight buffer, laid out
+// as a BF16 box arrives (rows of 128 bytes, 16-byte chunks swizzled by row & 7,
+// so the 32 rows of a warp's stores hit distinct banks).  Warp w owns weight
+// rows 32 (w % 4) .. + 31 of the unit (one row per thread) and one half of each
+// staging slot (warps 10..13 the second half): INT4 slot = two k-blocks (half h
+// -> k-block 2g + h, 32 code bytes -> 64 elements -> 8 chunks), INT8 slot = one
+// k-block (half h -> elements 32 h .. + 31 -> chunks 4 h .. 4 h + 3).
 template <bool kFma>
-__device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
+__device__ void dequant_swap(const Params& p, const Smem& s) {
   volatile int* abort_flag = s.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3;
   const int half = warp >= 10 ? 1 : 0;
-  const int r = quarter * 32 + lane;  // weight row of the unit = TMEM lane
-  const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + p.a_col;
+  const int r = quarter * 32 + lane;  // weight row of the unit
   const uint32_t ns = p.ns, nq = p.nq;
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
   uint32_t fph = 0;   // wfree phase bit per stage: INT8/INT4 tensor-core positions only
@@ -1413,7 +1402,6 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
       tr_wq += tq1 - tq0;
       tr_ww += tq2 - tq1;
       fph ^= (1u << st0) | (int4 ? 1u << st1 : 0u);
-      tc_fence_after();
       const uint4* src = reinterpret_cast<const uint4*>(s.q_st + q * s.qslot + r * 64 + half * 32);
       const uint4 c0 = src[0], c1 = src[1];
       const float sc = __half2float(reinterpret_cast<const __half*>(s.q_sc + q * s.qscale)[r]);
@@ -1428,7 +1416,11 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
           for (int b = 0; b < 4; ++b) v[4 * j + b] = deq2(lo, sel_byte(b), hi, sel_byte(b), s2, k2);
         }
         tr_conv += FFN_CLOCK() - tq2;
-        tmem_st32(lane_addr + (half ? st1 : st0) * 32, v);
+        const uint32_t row = smem_u32(s.w_st + (half ? st1 : st0) * s.wstage) + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(row + ((c ^ (r & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2],
+                       v[4 * c + 3]);
       } else {
         uint32_t v[16];  // word j = elements 4 j .. 4 j + 3 -> columns 2 j, 2 j + 1
 #pragma unroll
@@ -1438,11 +1430,16 @@ __device__ void dequant_tmem(const Params& p, const Smem& s, uint32_t tmem) {
           v[2 * j + 1] = deq2(a, sel_byte(2), a, sel_byte(3), s2, k2);
         }
         tr_conv += FFN_CLOCK() - tq2;
-        tmem_st16(lane_addr + st0 * 32 + half * 16, v);
+        const uint32_t row = smem_u32(s.w_st + st0 * s.wstage) + r * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int cc = half * 4 + c;
+          st_shared_v4(row + ((cc ^ (r & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2],
+                       v[4 * c + 3]);
+        }
       }
       const long long tq3 = FFN_CLOCK();
-      tmem_st_wait();
-      tc_fence_before();
+      fence_proxy_async_smem();  // the tensor core (async proxy) reads these bytes
       __syncwarp();
       if (lane == 0) {  // one arrival per dequant warp and stage
         mbar_arrive(&s.full[st0]);
@@ -1771,7 +1768,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) scheduler<kSwap, kFma>(p, s);
   } else {
     if (kSwap) {
-      dequant_tmem<kFma>(p, s, tmem);
+      dequant_swap<kFma>(p, s);
     } else {
       const int dtid = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // warps 2, 3, 8 .. 13
       dequant(p, s, dtid);

@@ -702,16 +702,13 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
   const int xbox = xrows;  // one X copy per stage
   const int nq = 4;
   // TMEM (512 columns): swap mode holds two accumulators of acc_stride columns
-  // (a power of two >= the token tile) and one 32-column A stage per operand
-  // stage; tile mode two 256-column accumulators.
+  // (a power of two >= the token tile), tile mode two of 256 columns.
   int acc_stride = 256;
   if (swap) {
     acc_stride = 16;
     while (acc_stride < xrows) acc_stride *= 2;
   }
-  const int a_col = swap ? 2 * acc_stride : 0;
-  const int ns_tmem = swap ? ((int)kTmemCols - a_col) / 32 : kMaxNS;
-  int ns = std::min(kMaxNS, ns_tmem);
+  int ns = kMaxNS;
   while (ns > 2 && (int)smem_map(swap, ns, nq, xrows, L->E).total > kSmemLimit) --ns;
   const int smem = (int)smem_map(swap, ns, nq, xrows, L->E).total;
   MOE_CHECK(smem <= kSmemLimit, MOE_ERR_UNSUPPORTED, "shared memory plan does not fit");
@@ -739,7 +736,7 @@ int grouped_ffn_impl(moe_layer_t L, const void* x_perm, const int32_t* expert_of
   Params prm{L->d_descs, L->d_prec, expert_offsets, h, static_cast<__nv_bfloat16*>(y_perm),
              counters, counters + 16, counters + 16 + L->E, rows, L->E, L->H, L->I,
              swap ? L->I / 64 : L->I / 128, swap ? L->H / 128 : (L->H + 255) / 256,
-             xbox, xrows, ns, nq, acc_stride, a_col, fma_rows};
+             xbox, xrows, ns, nq, acc_stride, fma_rows};
 
   rc = set_ffn_attributes(dev);
   if (rc != MOE_OK) return rc;
