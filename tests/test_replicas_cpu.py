@@ -34,7 +34,7 @@ def _max_worker(rank, world, port, out):
 
 def test_step_time_is_the_max_over_ranks():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of a threaded process
     mp.spawn(_max_worker, args=(world, port, out), nprocs=world, join=True)
     assert dict(out) == {0: 2.5, 1: 2.5}
 
