@@ -780,7 +780,23 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_h,
     for (int kb = 0; kb < nkb; ++kb) {
       if (kb == reserve_kb) mbar_arrive(s.go);
       const long long c0 = FFN_CLOCK();
-      if (!mbar_wait(&s.empty[st], sph ^ 1u, abort_flag)) {
+      bool freed;
+      if (kFma) {
+        // The stage's last use decides what frees it: the MMA commit on empty
+        // after a tensor-core position, all dequant warps' arrivals on fdone
+        // after a CUDA-core one.  Each barrier completes once per use of its
+        // kind, so the parity is that of the use-count bit (tc_par / fma_par).
+        const uint32_t bit = 1u << st;
+        if (!(issued & bit))
+          freed = true;  // never filled
+        else if (issued_fma & bit)
+          freed = mbar_wait(&s.fdone[st], ((fma_par >> st) & 1u) ^ 1u, abort_flag);
+        else
+          freed = mbar_wait(&s.empty[st], ((tc_par >> st) & 1u) ^ 1u, abort_flag);
+      } else {
+        freed = mbar_wait(&s.empty[st], sph ^ 1u, abort_flag);
+      }
+      if (!freed) {
         ok = false;
         break;
       }
@@ -1125,14 +1141,12 @@ __device__ __forceinline__ uint32_t nib_f32(uint32_t a, uint32_t b) {
 
 template <int N, bool kInt4, bool kHalf>
 __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const Unit& un, int ft,
-                                         uint32_t& st, uint32_t& sph, uint32_t& ffph,
-                                         uint32_t& fdph, Unit& pub, long long* tr) {
+                                         uint32_t& st, uint32_t& sph, uint32_t& ffph, Unit& pub,
+                                         long long* tr) {
   long long& tr_wait = tr[0];
   long long& tr_conv = tr[1];
-  long long& tr_sync = tr[2];
   long long& tr_out = tr[3];
   long long& tr_pub = tr[4];
-  (void)tr_sync;
   (void)tr_out;
   (void)tr_pub;
   volatile int* abort_flag = s.abort_flag;
@@ -1227,17 +1241,10 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
       }
     }
     tr_conv += FFN_CLOCK() - c1;
-    // Every dequant warp is done with the stage: thread 0 forwards the eight
-    // arrivals to the stage's empty barrier (the producer's refill condition).
+    // This warp is done with the stage; the producer refills it once all
+    // eight dequant warps have arrived (no warp waits for the others).
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.fdone[st]);
-    if (ft == 0) {
-      const long long c2 = FFN_CLOCK();
-      if (!mbar_wait(&s.fdone[st], (fdph >> st) & 1u, abort_flag)) return false;
-      tr_sync += FFN_CLOCK() - c2;
-      mbar_arrive(&s.empty[st]);
-    }
-    fdph ^= 1u << st;
     advance(st, sph, ns);
     // the previous gate/up unit's h rows, stored a stage ago: publishing them
     // now costs little (the fence no longer waits for stores in flight)
@@ -1283,17 +1290,16 @@ __device__ __forceinline__ bool fma_unit(const Params& p, const Smem& s, const U
 
 template <bool kInt4>
 __device__ bool fma_dispatch(const Params& p, const Smem& s, const Unit& un, int ft, uint32_t& st,
-                             uint32_t& sph, uint32_t& ffph, uint32_t& fdph, Unit& pub,
-                             long long* tr) {
+                             uint32_t& sph, uint32_t& ffph, Unit& pub, long long* tr) {
   static_assert(kFmaRows >= 1 && kFmaRows <= 2, "CUDA-core tiles of 1 or 2 rows");
   if (!unit_gu(un)) {  // down units: 64 weight rows
     if (kFmaRows >= 2 && un.nrows == 2)
-      return fma_unit<2, kInt4, true>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
-    return fma_unit<1, kInt4, true>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+      return fma_unit<2, kInt4, true>(p, s, un, ft, st, sph, ffph, pub, tr);
+    return fma_unit<1, kInt4, true>(p, s, un, ft, st, sph, ffph, pub, tr);
   }
   if (kFmaRows >= 2 && un.nrows == 2)
-    return fma_unit<2, kInt4, false>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
-  return fma_unit<1, kInt4, false>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+    return fma_unit<2, kInt4, false>(p, s, un, ft, st, sph, ffph, pub, tr);
+  return fma_unit<1, kInt4, false>(p, s, un, ft, st, sph, ffph, pub, tr);
 }
 
 // One staging slot holds an INT4 group (128 K-elements = two k-blocks) or an
@@ -1322,7 +1328,6 @@ __device__ void dequant_swap(const Params& p, const Smem& s) {
   uint32_t st = 0, sph = 0, q = 0, qph = 0, us = 0, uph = 0;
   uint32_t fph = 0;   // wfree phase bit per stage: INT8/INT4 tensor-core positions only
   uint32_t ffph = 0;  // ffull phase bit per stage: CUDA-core positions only
-  uint32_t fdph = 0;  // fdone phase bit per stage: CUDA-core positions only
   const int ft = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // warps 2, 3, 8 .. 13
   // A CUDA-core gate/up unit's h rows are published (fence + release add) one
   // stage into the next CUDA-core unit, when their stores have landed -- and
@@ -1362,8 +1367,8 @@ __device__ void dequant_swap(const Params& p, const Smem& s) {
     if (unit_fma<kFma>(un)) {
       long long tr[5] = {0, 0, 0, 0, 0};
       ok = un.prec == MOE_INT4
-               ? fma_dispatch<true>(p, s, un, ft, st, sph, ffph, fdph, pub, tr)
-               : fma_dispatch<false>(p, s, un, ft, st, sph, ffph, fdph, pub, tr);
+               ? fma_dispatch<true>(p, s, un, ft, st, sph, ffph, pub, tr)
+               : fma_dispatch<false>(p, s, un, ft, st, sph, ffph, pub, tr);
       if (!ok) break;
       if (tracer) {
         FFN_TRACE_SET(tseq, kTrDqEnd, FFN_TRACE_NS());
@@ -1718,9 +1723,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // producer's arrive.expect_tx, then one arrival per dequant warp (INT8/INT4
       // positions) or kDequantWarps more from the producer (BF16 positions)
       mbar_init(&s.full[i], 1 + kDequantWarps);
-      mbar_init(&s.empty[i], 1);               // tcgen05.commit, or dequant thread 0 (CUDA-core)
+      mbar_init(&s.empty[i], 1);               // tcgen05.commit (tensor-core positions)
       mbar_init(&s.wfree[i], 1);               // producer, at INT8/INT4 tensor-core positions
-      mbar_init(&s.fdone[i], kDequantWarps);   // each dequant warp, at CUDA-core positions
+      mbar_init(&s.fdone[i], kDequantWarps);   // each dequant warp (CUDA-core positions)
       mbar_init(&s.ffull[i], 1);               // producer's expect_tx, at CUDA-core positions
     } else if (i >= kMaxNS && i < kMaxNS + kMaxNQ) {
       mbar_init(&s.qfull[i - kMaxNS], 1);
