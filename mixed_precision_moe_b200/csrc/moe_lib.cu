@@ -828,7 +828,10 @@ int moe_combine(const void* y_perm, const int32_t* dest_row, const float* topk_w
   MOE_CHECK(aligned(y_perm, 16) && aligned(out, 16), MOE_ERR_UNSUPPORTED,
             "y_perm and out must be 16-byte aligned");
   const int vec = H / 8;
-  const dim3 block(std::min(256, ((vec + 31) / 32) * 32));
+  // decode-sized batches: 64-thread blocks, so a token's row is spread over
+  // more SMs and more of its loads are in flight at once
+  const int bmax = T <= 128 ? 64 : 256;
+  const dim3 block(std::min(bmax, ((vec + 31) / 32) * 32));
   const dim3 grid(T, (vec + block.x - 1) / block.x);
   MOE_CUDA_TRY(launch_pdl(moe::combine_kernel, grid, block, 0, as_stream(stream),
                           static_cast<const uint4*>(y_perm), dest_row, topk_w, k, vec, T * k,

@@ -478,6 +478,9 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 // grid (T, ceil(H/8 / blockDim.x)); each thread one 16-byte vector of a row.
 // Pairs with dest_row < 0 are skipped; a row >= rows (the capacity of y,
 // T * k) is skipped too and flagged, so no read leaves y.
+// The k row indices and weights are loaded first, then all k vectors, and only
+// then summed (same order as above): two dependent memory round trips per
+// token instead of k, which at decode sizes is most of the kernel's time.
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y,
                                                       const int32_t* __restrict__ dest_row,
                                                       const float* __restrict__ topk_w, int k,
@@ -488,19 +491,36 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   const int t = blockIdx.x;
   const int c = blockIdx.y * blockDim.x + threadIdx.x;
   if (c >= vec_per_row) return;
+  constexpr int kMaxK = 16;  // the host rejects k > 16
+  int r[kMaxK];
+  float wt[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    r[j] = -1;
+    wt[j] = 0.0f;
+    if (j < k) {
+      r[j] = dest_row[(size_t)t * k + j];
+      wt[j] = topk_w[(size_t)t * k + j];
+    }
+  }
+  uint4 v[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    v[j] = make_uint4(0u, 0u, 0u, 0u);
+    if (r[j] >= 0 && r[j] < rows) v[j] = y[(size_t)r[j] * vec_per_row + c];
+  }
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int j = 0; j < k; ++j) {
-    const int r = dest_row[(size_t)t * k + j];
-    if (r < 0) continue;
-    if (r >= rows) {
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    if (r[j] < 0) continue;
+    if (r[j] >= rows) {
       if (c == 0) flag_status(MOE_STATUS_BAD_ROW_INDEX);
       continue;
     }
-    const float wj = topk_w[(size_t)t * k + j];
     float f[8];
-    bf16x8_to_f32(y[(size_t)r * vec_per_row + c], f);
+    bf16x8_to_f32(v[j], f);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+    for (int i = 0; i < 8; ++i) acc[i] = fmaf(wt[j], f[i], acc[i]);
   }
   uint4 o;
   o.x = pack_bf16x2(acc[0], acc[1]);
